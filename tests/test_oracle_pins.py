@@ -1,0 +1,402 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Each check ties the oracle to something the pages or mathematics fix: a
+library attention routine in fp64, brute force on tiny inputs, closed forms,
+invariants, hand-derived worked examples (tests/golden/), and planted mistakes
+that at least one pin must catch.  The definition checked is the one in the
+header of oracle/pba_oracle.c (pair-biased attention, "Fold-CP: A Context
+Parallelism Framework for Biomolecular Modeling", Table 1 and Figure 2).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def _num(x):
+    if isinstance(x, str):
+        return float(x)
+    if isinstance(x, list):
+        return [_num(y) for y in x]
+    return x
+
+
+def _rand_problem(B=2, H=3, Nq=37, Nk=53, D=16, seed=0, mask_frac=0.2, neg_inf_frac=0.0, bias_std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, H, Nq, D, generator=g, dtype=torch.float64)
+    k = torch.randn(B, H, Nk, D, generator=g, dtype=torch.float64)
+    v = torch.randn(B, H, Nk, D, generator=g, dtype=torch.float64)
+    bias = torch.randn(B, H, Nq, Nk, generator=g, dtype=torch.float64) * bias_std
+    if neg_inf_frac > 0:
+        bias[torch.rand(B, H, Nq, Nk, generator=g) < neg_inf_frac] = -math.inf
+    mask = (torch.rand(B, Nk, generator=g) >= mask_frac).to(torch.uint8) if mask_frac > 0 else None
+    return q, k, v, bias, mask
+
+
+def _sdpa_reference(q, k, v, bias, mask):
+    """torch's math-path scaled_dot_product_attention in fp64 with the bias
+    and the key mask as an additive float mask."""
+    add = bias.clone()
+    if mask is not None:
+        add = add + torch.where(mask.bool(), 0.0, -math.inf).to(torch.float64)[:, None, None, :]
+    with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=add)
+    scores = torch.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(q.shape[-1]) + add
+    lse = torch.logsumexp(scores, dim=-1)
+    return o, lse, torch.isinf(lse)
+
+
+# ---------------------------------------------------------------- library
+@pytest.mark.parametrize("D", [4, 16, 32, 64])
+@pytest.mark.parametrize("seed", [0, 1])
+def test_matches_torch_sdpa_fp64(D, seed):
+    q, k, v, bias, mask = _rand_problem(D=D, seed=seed, neg_inf_frac=0.05)
+    r = oracle.pba(q, k, v, bias, mask)
+    o_ref, lse_ref, empty = _sdpa_reference(q, k, v, bias, mask)
+    keep = ~empty
+    assert np.abs(r["o"][keep.numpy()] - o_ref[keep].numpy()).max() < 1e-12
+    assert np.abs(r["lse"][keep.numpy()] - lse_ref[keep].numpy()).max() < 1e-12
+
+
+def test_matches_torch_sdpa_fp64_n512():
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=512, Nk=512, D=32, seed=7, mask_frac=0.1)
+    r = oracle.pba(q, k, v, bias, mask)
+    o_ref, lse_ref, _ = _sdpa_reference(q, k, v, bias, mask)
+    assert np.abs(r["o"] - o_ref.numpy()).max() < 1e-12
+    assert np.abs(r["lse"] - lse_ref.numpy()).max() < 1e-12
+
+
+# ---------------------------------------------------------------- brute force
+def _brute_force(q, k, v, bias, mask):
+    """Pure-Python loops, no max subtraction, math.fsum for the sums."""
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    tau = 1.0 / math.sqrt(D)
+    o = np.zeros((B, H, Nq, D))
+    lse = np.zeros((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            for i in range(Nq):
+                w = []
+                for j in range(Nk):
+                    if mask is not None and mask[b, j] == 0:
+                        continue
+                    bij = float(bias[b, h, i, j])
+                    if bij == -math.inf:
+                        continue
+                    s = tau * math.fsum(float(q[b, h, i, d]) * float(k[b, h, j, d]) for d in range(D)) + bij
+                    w.append((math.exp(s), j))
+                if not w:
+                    lse[b, h, i] = -math.inf
+                    continue
+                Z = math.fsum(e for e, _ in w)
+                lse[b, h, i] = math.log(Z)
+                for d in range(D):
+                    o[b, h, i, d] = math.fsum(e * float(v[b, h, j, d]) for e, j in w) / Z
+    return o, lse
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_brute_force_tiny(seed):
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=7, Nk=16, D=8, seed=seed, mask_frac=0.25, neg_inf_frac=0.1)
+    r = oracle.pba(q, k, v, bias, mask)
+    o_bf, lse_bf = _brute_force(q.numpy(), k.numpy(), v.numpy(), bias.numpy(), None if mask is None else mask.numpy())
+    assert np.allclose(r["o"], o_bf, atol=1e-12, rtol=0)
+    fin = np.isfinite(lse_bf)
+    assert np.array_equal(fin, np.isfinite(r["lse"]))
+    assert np.abs(r["lse"][fin] - lse_bf[fin]).max() < 1e-12
+
+
+# ---------------------------------------------------------------- invariants and closed forms
+def test_rows_sum_to_one():
+    q, k, v, bias, mask = _rand_problem(seed=3, mask_frac=0.3)
+    r = oracle.pba(q, k, torch.ones_like(v), bias, mask)
+    assert np.abs(r["o"] - 1.0).max() < 1e-14
+
+
+def test_shift_invariance_per_row():
+    q, k, v, bias, mask = _rand_problem(seed=4, mask_frac=0.1)
+    c = torch.randn(bias.shape[:-1], dtype=torch.float64, generator=torch.Generator().manual_seed(9)) * 5
+    r0 = oracle.pba(q, k, v, bias, mask)
+    r1 = oracle.pba(q, k, v, bias + c[..., None], mask)
+    assert np.abs(r0["o"] - r1["o"]).max() < 1e-12
+    assert np.abs((r0["lse"] + c.numpy()) - r1["lse"]).max() < 1e-12
+
+
+def test_zero_q_zero_bias_gives_mean_of_valid_values():
+    q, k, v, bias, mask = _rand_problem(seed=5, mask_frac=0.4)
+    r = oracle.pba(torch.zeros_like(q), k, v, torch.zeros_like(bias), mask)
+    mk = mask.numpy().astype(bool)
+    for b in range(q.shape[0]):
+        n_valid = mk[b].sum()
+        mean = v[b][:, mk[b]].numpy().mean(axis=1)  # [H, D]
+        assert np.abs(r["o"][b] - mean[:, None, :]).max() < 1e-13
+        assert np.abs(r["lse"][b] - math.log(n_valid)).max() < 1e-13
+        assert np.abs(r["l"][b] - n_valid).max() < 1e-12 and np.all(r["m"][b] == 0.0)
+
+
+def test_one_hot_bias_closed_form():
+    Nk, D = 20, 8
+    q, k, v, bias, _ = _rand_problem(B=1, H=1, Nq=3, Nk=Nk, D=D, seed=6, mask_frac=0)
+    bias = torch.zeros_like(bias)
+    jstar = 11
+    bias[..., jstar] = 30.0
+    r = oracle.pba(torch.zeros_like(q), k, v, bias)
+    e = math.exp(-30.0)
+    vv = v[0, 0].numpy()
+    expect = (vv[jstar] + e * (vv.sum(axis=0) - vv[jstar])) / (1.0 + (Nk - 1) * e)
+    assert np.abs(r["o"][0, 0] - expect[None, :]).max() < 1e-14
+    assert abs(r["lse"][0, 0, 0] - (30.0 + math.log1p((Nk - 1) * e))) < 1e-14
+
+
+def test_single_key():
+    q, k, v, bias, _ = _rand_problem(B=1, H=2, Nq=5, Nk=1, D=8, seed=7, mask_frac=0)
+    r = oracle.pba(q, k, v, bias)
+    assert np.abs(r["o"] - v.numpy()).max() == 0.0
+    s0 = (q * k).sum(-1).numpy() / math.sqrt(8) + bias[..., 0].numpy()
+    assert np.abs(r["lse"] - s0).max() < 1e-14
+
+
+def test_fully_masked_rows():
+    q, k, v, bias, _ = _rand_problem(B=1, H=2, Nq=4, Nk=9, D=8, seed=8, mask_frac=0)
+    bias[0, 1, 2, :] = -math.inf
+    mask = torch.ones(1, 9, dtype=torch.uint8)
+    r = oracle.pba(q, k, v, bias, mask)
+    assert np.all(r["o"][0, 1, 2] == 0.0) and r["lse"][0, 1, 2] == -math.inf
+    assert r["m"][0, 1, 2] == -math.inf and r["l"][0, 1, 2] == 0.0
+    r = oracle.pba(q, k, v, bias, torch.zeros(1, 9, dtype=torch.uint8))
+    assert np.all(r["o"] == 0.0) and np.all(r["lse"] == -math.inf) and np.all(r["l"] == 0.0)
+
+
+def test_permutations_and_head_independence():
+    q, k, v, bias, mask = _rand_problem(seed=10, mask_frac=0.2)
+    r0 = oracle.pba(q, k, v, bias, mask)
+    g = torch.Generator().manual_seed(11)
+    pk = torch.randperm(k.shape[2], generator=g)
+    r1 = oracle.pba(q, k[:, :, pk], v[:, :, pk], bias[..., pk], mask[:, pk])
+    assert np.abs(r0["o"] - r1["o"]).max() < 1e-13
+    pq = torch.randperm(q.shape[2], generator=g)
+    r2 = oracle.pba(q[:, :, pq], k, v, bias[:, :, pq], mask)
+    assert np.abs(r0["o"][:, :, pq.numpy()] - r2["o"]).max() == 0.0
+    q2 = q.clone()
+    q2[:, 1] += 1.0
+    r3 = oracle.pba(q2, k, v, bias, mask)
+    assert np.array_equal(r0["o"][:, 0], r3["o"][:, 0]) and np.array_equal(r0["o"][:, 2], r3["o"][:, 2])
+    assert np.abs(r0["o"][:, 1] - r3["o"][:, 1]).max() > 1e-3
+
+
+# ---------------------------------------------------------------- partials and merge
+@pytest.mark.parametrize("seed", range(5))
+def test_merge_of_random_chunkings_equals_single_pass(seed):
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=9, Nk=61, D=8, seed=20 + seed, mask_frac=0.3,
+                                        neg_inf_frac=0.05)
+    full = oracle.pba(q, k, v, bias, mask)
+    rng = np.random.default_rng(seed)
+    Nk = k.shape[2]
+    cuts = sorted(set(rng.integers(1, Nk, size=rng.integers(0, 8)).tolist()))
+    edges = [0] + cuts + [Nk]
+    blocks = list(zip(edges[:-1], edges[1:]))
+    order = rng.permutation(len(blocks))
+    parts = [oracle.pba_partial(q, k, v, bias, mask, k0=blocks[p][0], L=blocks[p][1] - blocks[p][0]) for p in order]
+    o_parts = np.stack([p["o"] for p in parts])
+    m_parts = np.stack([p["m"] for p in parts])
+    l_parts = np.stack([p["l"] for p in parts])
+    mrg = oracle.merge(o_parts, m_parts, l_parts)
+    assert np.abs(mrg["o"] - full["o"]).max() < 1e-12
+    fin = np.isfinite(full["lse"])
+    assert np.array_equal(fin, np.isfinite(mrg["lse"]))
+    assert np.abs(mrg["lse"][fin] - full["lse"][fin]).max() < 1e-12
+
+
+def test_merge_identities():
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=6, Nk=30, D=8, seed=30, mask_frac=0.2)
+    part = oracle.pba_partial(q, k, v, bias, mask, k0=0, L=30)
+    full = oracle.pba(q, k, v, bias, mask)
+    one = oracle.merge(part["o"][None], part["m"][None], part["l"][None])
+    assert np.abs(one["o"] - full["o"]).max() < 1e-14 and np.abs(one["lse"] - full["lse"]).max() < 1e-14
+    empty_o = np.zeros_like(part["o"])
+    empty_m = np.full_like(part["m"], -np.inf)
+    empty_l = np.zeros_like(part["l"])
+    two = oracle.merge(np.stack([empty_o, part["o"]]), np.stack([empty_m, part["m"]]), np.stack([empty_l, part["l"]]))
+    assert np.abs(two["o"] - full["o"]).max() < 1e-14 and np.abs(two["lse"] - full["lse"]).max() < 1e-14
+    # a block with no valid key is exactly (0, -inf, 0)
+    allmask = torch.zeros_like(mask)
+    e = oracle.pba_partial(q, k, v, bias, allmask, k0=5, L=10)
+    assert np.all(e["o"] == 0.0) and np.all(e["m"] == -np.inf) and np.all(e["l"] == 0.0)
+
+
+def test_partial_block_sum_matches_brute_force():
+    q, k, v, bias, mask = _rand_problem(B=1, H=1, Nq=5, Nk=16, D=8, seed=31, mask_frac=0.2)
+    p = oracle.pba_partial(q, k, v, bias, mask, k0=4, L=7)
+    sl = slice(4, 11)
+    o_bf, lse_bf = _brute_force(q.numpy(), k[:, :, sl].numpy(), v[:, :, sl].numpy(), bias[..., sl].numpy(),
+                                mask[:, sl].numpy())
+    assert np.abs(p["o"] - o_bf).max() < 1e-12
+    fin = np.isfinite(lse_bf)
+    assert np.abs((p["m"] + np.log(p["l"]))[fin] - lse_bf[fin]).max() < 1e-12
+
+
+# ---------------------------------------------------------------- triangle attention
+def _tri_problem(N=12, H=2, D=8, seed=40, mask_frac=0.2):
+    g = torch.Generator().manual_seed(seed)
+    q, k, v, gt = (torch.randn(N, N, H, D, generator=g, dtype=torch.float64) for _ in range(4))
+    bias = torch.randn(H, N, N, generator=g, dtype=torch.float64)
+    pm = (torch.rand(N, N, generator=g) >= mask_frac).to(torch.uint8) if mask_frac > 0 else None
+    return q, k, v, gt, bias, pm
+
+
+def _tri_einsum(q, k, v, g, bias, pm, ending):
+    """fp64 restatement with torch.einsum and torch.softmax (N <= 32)."""
+    D = q.shape[-1]
+    if not ending:
+        s = torch.einsum("ijhd,ikhd->ijhk", q, k) / math.sqrt(D) + bias.permute(1, 0, 2)[None]  # b[h][j][k]
+        if pm is not None:
+            s = s + torch.where(pm.bool(), 0.0, -math.inf).double()[:, None, None, :]
+        a = torch.softmax(s, dim=-1)
+        o = torch.einsum("ijhk,ikhd->ijhd", a, v)
+    else:
+        s = torch.einsum("ijhd,kjhd->ijhk", q, k) / math.sqrt(D) + bias.permute(2, 0, 1)[:, None]  # b[h][k][i]
+        if pm is not None:
+            s = s + torch.where(pm.bool(), 0.0, -math.inf).double().t()[None, :, None, :]
+        a = torch.softmax(s, dim=-1)
+        o = torch.einsum("ijhk,kjhd->ijhd", a, v)
+    lse = torch.logsumexp(s, dim=-1)
+    return o * torch.sigmoid(g), lse
+
+
+@pytest.mark.parametrize("ending", [False, True])
+def test_tri_matches_einsum_restatement(ending):
+    q, k, v, g, bias, pm = _tri_problem()
+    r = oracle.tri_attn(q, k, v, bias, g, pm, ending=ending)
+    o_ref, lse_ref = _tri_einsum(q, k, v, g, bias, pm, ending)
+    if ending:  # line layout: line l = column j
+        o_ref, lse_ref = o_ref.transpose(0, 1), lse_ref.transpose(0, 1)
+    assert np.abs(r["o"] - o_ref.numpy()).max() < 1e-12
+    assert np.abs(r["lse"] - lse_ref.numpy()).max() < 1e-12
+
+
+def test_tri_starting_row_is_pair_biased_attention():
+    q, k, v, g, bias, pm = _tri_problem(mask_frac=0.2)
+    r = oracle.tri_attn(q, k, v, bias, None, pm, ending=False)
+    for i in (0, 5, 11):
+        # row i: queries j, keys k of head h -> [1, H, N, D]
+        pr = oracle.pba(q[i].permute(1, 0, 2)[None], k[i].permute(1, 0, 2)[None], v[i].permute(1, 0, 2)[None],
+                        bias[None], pm[i][None])
+        assert np.abs(r["o"][i] - pr["o"][0].transpose(1, 0, 2)).max() < 1e-13
+        assert np.abs(r["lse"][i] - pr["lse"][0].T).max() < 1e-13
+
+
+def test_tri_ending_equals_starting_on_transpose():
+    q, k, v, g, bias, pm = _tri_problem(mask_frac=0.2)
+    end = oracle.tri_attn(q, k, v, bias, g, pm, ending=True)  # line l = column j
+    T = lambda x: x.transpose(0, 1).contiguous()
+    st = oracle.tri_attn(T(q), T(k), T(v), bias.transpose(1, 2).contiguous(), T(g), pm.t().contiguous(),
+                         ending=False)  # line l = row l of the transpose = column l of the original
+    assert np.abs(end["o"] - st["o"]).max() < 1e-13
+    assert np.abs(end["lse"] - st["lse"]).max() < 1e-13
+
+
+# ---------------------------------------------------------------- golden worked examples
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+@pytest.mark.parametrize("case", _golden()["attention"], ids=lambda c: c["name"])
+def test_golden_attention(case):
+    t = lambda x: torch.tensor(_num(x), dtype=torch.float64)[None, None]
+    mask = None if case["key_mask"] is None else torch.tensor(case["key_mask"], dtype=torch.uint8)[None]
+    r = oracle.pba(t(case["q"]), t(case["k"]), t(case["v"]), t(case["bias"]), mask)
+    assert np.abs(r["o"][0, 0] - np.array(_num(case["o"]))).max() < 1e-14
+    for key in ("lse", "m", "l"):
+        exp = np.array(_num(case[key]))
+        got = r[key][0, 0]
+        assert np.array_equal(np.isfinite(exp), np.isfinite(got))
+        fin = np.isfinite(exp)
+        assert np.all(exp[~fin] == got[~fin])
+        assert np.abs(got[fin] - exp[fin]).max(initial=0.0) < 1e-14
+
+
+@pytest.mark.parametrize("case", _golden()["merge"], ids=lambda c: c["name"])
+def test_golden_merge(case):
+    r = oracle.merge(np.array(_num(case["o_parts"])), np.array(_num(case["m_parts"])), np.array(_num(case["l_parts"])))
+    assert np.abs(r["o"] - np.array(_num(case["o"]))).max() < 1e-14
+    assert np.abs(r["lse"] - np.array(_num(case["lse"]))).max() < 1e-14
+
+
+@pytest.mark.parametrize("case", _golden()["triangle"], ids=lambda c: c["name"])
+@pytest.mark.parametrize("gate", [False, True])
+def test_golden_triangle(case, gate):
+    bias = torch.tensor(_num(case["bias"]), dtype=torch.float64)
+    v = torch.tensor(_num(case["v"]), dtype=torch.float64)
+    z = torch.zeros_like(v)
+    g = z if gate else None
+    scale = 0.5 if gate else 1.0
+    st = oracle.tri_attn(z, z, v, bias, g, None, ending=False)
+    en = oracle.tri_attn(z, z, v, bias, g, None, ending=True)
+    assert np.abs(st["o"] - scale * np.array(case["starting_o"])).max() < 1e-14
+    assert np.abs(st["lse"] - np.array(case["starting_lse"])).max() < 1e-14
+    # ending-node lines are columns: transpose back to [i][j]
+    assert np.abs(en["o"].transpose(1, 0, 2, 3) - scale * np.array(case["ending_o"])).max() < 1e-14
+    assert np.abs(en["lse"].transpose(1, 0, 2) - np.array(case["ending_lse"])).max() < 1e-14
+
+
+# ---------------------------------------------------------------- planted mistakes
+def _pin_suite(mutant):
+    """Run a compact set of the pins against an oracle build; return the
+    number that fail."""
+    fails = 0
+    gold = _golden()
+    t = lambda x: torch.tensor(_num(x), dtype=torch.float64)[None, None]
+    for case in gold["attention"]:
+        mask = None if case["key_mask"] is None else torch.tensor(case["key_mask"], dtype=torch.uint8)[None]
+        r = oracle.pba(t(case["q"]), t(case["k"]), t(case["v"]), t(case["bias"]), mask, mutant=mutant)
+        exp_lse = np.array(_num(case["lse"]))
+        fin = np.isfinite(exp_lse)
+        if (np.abs(r["o"][0, 0] - np.array(_num(case["o"]))).max() > 1e-12
+                or np.abs(r["lse"][0, 0][fin] - exp_lse[fin]).max(initial=0) > 1e-12):
+            fails += 1
+    for case in gold["merge"]:
+        r = oracle.merge(np.array(_num(case["o_parts"])), np.array(_num(case["m_parts"])),
+                         np.array(_num(case["l_parts"])), mutant=mutant)
+        if np.abs(r["o"] - np.array(_num(case["o"]))).max() > 1e-12:
+            fails += 1
+    case = gold["triangle"][0]
+    bias = torch.tensor(_num(case["bias"]), dtype=torch.float64)
+    v = torch.tensor(_num(case["v"]), dtype=torch.float64)
+    z = torch.zeros_like(v)
+    en = oracle.tri_attn(z, z, v, bias, z, None, ending=True, mutant=mutant)
+    if np.abs(en["o"].transpose(1, 0, 2, 3) - 0.5 * np.array(case["ending_o"])).max() > 1e-12:
+        fails += 1
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=9, Nk=40, D=8, seed=21, mask_frac=0.2)
+    full = oracle.pba(q, k, v, bias, mask, mutant=0)
+    parts = [oracle.pba_partial(q, k, v, bias, mask, k0=a, L=b - a, mutant=mutant) for a, b in ((20, 40), (0, 7), (7, 20))]
+    mrg = oracle.merge(np.stack([p["o"] for p in parts]), np.stack([p["m"] for p in parts]),
+                       np.stack([p["l"] for p in parts]), mutant=mutant)
+    if np.abs(mrg["o"] - full["o"]).max() > 1e-10:
+        fails += 1
+    q, k, v, bias, mask = _rand_problem(seed=0, neg_inf_frac=0.05)
+    r = oracle.pba(q, k, v, bias, mask, mutant=mutant)
+    o_ref, lse_ref, empty = _sdpa_reference(q, k, v, bias, mask)
+    keep = (~empty).numpy()
+    if np.abs(r["o"][keep] - o_ref.numpy()[keep]).max() > 1e-10:
+        fails += 1
+    return fails
+
+
+def test_default_build_passes_compact_pins():
+    assert _pin_suite(0) == 0
+
+
+@pytest.mark.parametrize("mutant", range(1, 10))
+def test_planted_mistake_is_caught(mutant):
+    assert _pin_suite(mutant) > 0, f"planted mistake {mutant} went unnoticed"
