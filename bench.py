@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the pair-biased attention hot path on B200.
+
+One step = the "large" workload: pba_forward at N=16384, H=16, D=64 bf16 with a
+5% random key mask (bias [H,N,N] = 8.6 GB), then triangle attention on a pair
+tensor of N=1024, H=4, D=32 in both orientations.  Inputs are synthetic and
+seeded (workloads.py) and resident in HBM before the timed region; every input
+is larger than L2, so no flush is needed between iterations.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs the same
+workload on its own GPU (weak scaling, no collective on the data path); the
+step time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "pair-bias attention TFLOP/s & bias HBM GB/s vs roofline at N=16K; tri-attn rows/s"
+UNIT = "TFLOP/s"
+
+
+def attn_flops(B, H, Nq, Nk, D) -> float:
+    """Q K^T and P V: 2 * 2 * B*H*Nq*Nk*D (Fold-CP Table 1 serial time B H N^2 D)."""
+    return 4.0 * B * H * Nq * Nk * D
+
+
+def attn_bytes(B, H, Nq, Nk, D, elt=2, mask=True) -> float:
+    """Algorithmic HBM bytes of one pass: bias, Q, K, V read once, O and the
+    log-sum-exp written once, the key mask read once."""
+    return (B * H * Nq * Nk * elt + B * H * (Nq + 2 * Nk) * D * elt + B * H * Nq * D * elt + B * H * Nq * 4 +
+            (B * Nk if mask else 0))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid).replace("-", "").lower()
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            uid = parts[0].replace("GPU-", "").replace("-", "").lower()
+            if self.uuid and self.uuid not in uid and uid not in self.uuid:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        loaded = [s for s, p in zip(sm, power) if p > 300] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = False
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = True
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local, pg
+
+
+def max_over_ranks(x: float, pg: bool) -> float:
+    if not pg:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg: bool):
+    torch.cuda.synchronize()
+    if pg:
+        import torch.distributed as dist
+
+        dist.barrier()
+        torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_sample(q, k, v, bias, mask, target_s=10.0, max_rows=4096):
+    """Times the fp64 oracle on a bounded sample of query rows of the large
+    workload (all 16384 keys each).  Returns (TFLOP/s, threads, description)."""
+    import oracle
+
+    H, N, D = q.shape[1], q.shape[2], q.shape[3]
+    g = torch.Generator("cpu").manual_seed(77)
+
+    def run(nrows):
+        per_head = max(1, nrows // H)
+        flops, t = 0.0, 0.0
+        for h in range(H):
+            rows = torch.randperm(N, generator=g)[:per_head].to(q.device)
+            qs = q[:, h:h + 1].index_select(2, rows).cpu()
+            bs = bias[:, h:h + 1].index_select(2, rows).cpu()
+            ks, vs = k[:, h:h + 1].cpu(), v[:, h:h + 1].cpu()
+            ms = None if mask is None else mask.cpu()
+            t0 = time.perf_counter()
+            oracle.pba(qs, ks, vs, bs, ms)
+            t += time.perf_counter() - t0
+            flops += attn_flops(1, 1, per_head, N, D)
+        return flops, t, per_head * H
+
+    f, t, n = run(H * 4)
+    rate = f / t
+    want = int(min(max_rows, max(H, target_s * rate / attn_flops(1, 1, 1, N, D))))
+    f, t, n = run(want)
+    return f / t / 1e12, oracle.threads_used(), f"{n} query rows x {N} keys of large16k (fp64 oracle, sampled rows)", t
+
+
+# ------------------------------------------------------------------ the reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import oracle
+
+    oracle.build()
+    cfg = W.LARGE16K
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    q, k, v, bias, mask = W.attn_inputs(cfg, dev)
+    # each step runs the oracle on a bounded sample of rows of this workload
+    H, N, D = cfg.H, cfg.N, cfg.D
+    per_head = max(1, args.ref_rows // H)
+    g = torch.Generator("cpu").manual_seed(5)
+    sample = []
+    for h in range(H):
+        rows = torch.randperm(N, generator=g)[:per_head].to(q.device)
+        sample.append((q[:, h:h + 1].index_select(2, rows).cpu(), k[:, h:h + 1].cpu(), v[:, h:h + 1].cpu(),
+                       bias[:, h:h + 1].index_select(2, rows).cpu(), mask.cpu()))
+    del q, k, v, bias
+    flops_step = attn_flops(1, H, per_head, N, D)
+    for _ in range(args.warmup):
+        for s in sample[:1]:
+            oracle.pba(*s)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        for s in sample:
+            oracle.pba(*s)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = flops_step * args.steps / total / 1e12
+    cores = oracle.threads_used()
+    desc = f"{per_head * H} query rows x {N} keys of large16k per step (fp64 oracle)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "large16k: pair-biased attention N=16384 H=16 D=64, 5% random key mask (sampled rows)",
+                   "B": 1, "N": N, "H": H, "D": D},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512"], default="none",
+                    help="run one small case only (for ncu captures); prints no JSON line")
+    args = ap.parse_args()
+    world, rank, local, pg = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import pair_biased_attention_b200 as pba
+
+    pba.load_library()
+    dev = torch.device("cuda", local)
+
+    if args.profile != "none":
+        return run_profile_case(args, pba, dev)
+
+    peaks = load_peaks()
+    cfg = W.LARGE16K
+    tcfg = W.TRI1024
+    q, k, v, bias, mask = W.attn_inputs(cfg, dev)
+    tq, tk, tv, tg, tb = W.tri_inputs(tcfg, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.H, cfg.N), dtype=torch.float32, device=dev)
+    tout = torch.empty_like(tq)
+    tlse = torch.empty((tcfg.N, tcfg.N, tcfg.H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        pba.pba_forward(q, k, v, bias, mask, out, lse, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        pba.tri_attn_forward(tq, tk, tv, tb, tg, None, "starting", tout, tlse, stream=stream)
+        pba.tri_attn_forward(tq, tk, tv, tb, tg, None, "ending", tout, tlse, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    assert pba.pba_last_device_error(stream) == pba.PBA_OK
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    barrier(pg)
+    clocks.start()
+    for i in range(args.steps):
+        step(evs[i])
+    barrier(pg)
+    clk = clocks.stop()
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("a kernel recorded a device error during the timed steps")
+    pba_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    tri_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    t_pba = max_over_ranks(sum(pba_ms), pg)
+    t_tri = max_over_ranks(sum(tri_ms), pg)
+    t_step = max_over_ranks(sum(step_ms), pg)
+
+    flops = attn_flops(cfg.B, cfg.H, cfg.N, cfg.N, cfg.D)
+    nbytes = attn_bytes(cfg.B, cfg.H, cfg.N, cfg.N, cfg.D)
+    value = world * flops * args.steps / (t_pba / 1e3) / 1e12
+    avg_launch_s = sum(pba_ms) / len(pba_ms) / 1e3
+    achieved_gbs = nbytes / avg_launch_s / 1e9
+    tri_rows = 2 * tcfg.N  # pair-tensor rows per step (starting + ending)
+    tri_rows_per_s = world * tri_rows * args.steps / (t_tri / 1e3)
+    tri_flops = 2 * attn_flops(tcfg.N, tcfg.H, tcfg.N, tcfg.N, tcfg.D)
+
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("pba_attn_sm100_large16k_bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": t_step / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "large16k: pair-biased attention N=16384 H=16 D=64 bf16, bias [H,N,N] ~N(0,1), "
+                               "5% random key mask; plus triangle attention N=1024 c=128 H=4 D=32 (starting+ending)",
+                   "B": cfg.B, "N": cfg.N, "H": cfg.H, "D": cfg.D, "tri_N": tcfg.N, "tri_H": tcfg.H, "tri_D": tcfg.D,
+                   "l2": "no flush: every input is larger than L2 (bias 8.6 GB, tri q/k/v/g 1.07 GB)",
+                   "parallelism": f"replicas x{world} (independent problems per GPU)"},
+        "pba_ms_per_launch": sum(pba_ms) / len(pba_ms),
+        "bias_hbm_gbs": cfg.B * cfg.H * cfg.N * cfg.N * 2 / avg_launch_s / 1e9,
+        "tri_attn_rows_per_s": tri_rows_per_s,
+        "tri_attn_ms_per_call": sum(tri_ms) / len(tri_ms) / 2,
+        "tri_attn_tflops": world * tri_flops * args.steps / (t_tri / 1e3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": "pba_attn_sm100_kernel (pba_forward, large16k)",
+                     "algorithmic_bytes_per_launch": nbytes, "peak_source": peaks["source"],
+                     "tensor_frac": (flops / avg_launch_s / 1e12) / peaks["bf16_tflops_sustained"]},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
+    if not args.no_cpu and rank == 0 and world == 1:
+        val, cores, desc, secs = oracle_sample(q, k, v, bias, mask, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+                                "seconds": secs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops):
+    """Same metric through the public call with the inputs starting in pinned
+    host memory and the outputs read back each step."""
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hb = torch.empty(bias.shape, dtype=bias.dtype, pin_memory=True)
+    hb.copy_(bias)
+    hm = mask.cpu().pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hb, hm))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        bias.copy_(hb, non_blocking=True)
+        mask.copy_(hm, non_blocking=True)
+        pba.pba_forward(q, k, v, bias, mask, out, lse, stream=stream)
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    barrier(pg)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e.record(stream)
+    barrier(pg)
+    t = max_over_ranks(s.elapsed_time(e), pg)
+    assert torch.isfinite(hl[hl > -math.inf]).all()
+    return {"value": world * flops * args.e2e_steps / (t / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+def run_profile_case(args, pba, dev):
+    """One small case for ncu: pba4k = pba_forward at N=4096 (bias 512 MB,
+    larger than L2) after one warm-up launch; tri512 = triangle attention
+    N=512 both orientations."""
+    if args.profile == "pba4k":
+        cfg = W.AttnConfig("pba4k", B=1, N=4096, H=16, D=64, dtype=torch.bfloat16, seed=4, mask="random5")
+        q, k, v, bias, mask = W.attn_inputs(cfg, dev)
+        for _ in range(2):
+            pba.pba_forward(q, k, v, bias, mask)
+    else:
+        q, k, v, g, b = W.tri_inputs(W.TRI512, dev)
+        for _ in range(2):
+            pba.tri_attn_forward(q, k, v, b, g, None, "starting")
+            pba.tri_attn_forward(q, k, v, b, g, None, "ending")
+    torch.cuda.synchronize()
+    assert pba.pba_last_device_error() == pba.PBA_OK
+    print(f"profile case {args.profile} done")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

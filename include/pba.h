@@ -1,0 +1,204 @@
+/*
+ * pba.h -- C ABI of libpba: pair-biased attention on NVIDIA B200 (sm_100a).
+ *
+ * The operation (all entry points): multi-head attention whose logits carry
+ * an additive pair bias,
+ *
+ *     O = softmax_keys( tau * Q K^T + bias + mask ) V ,   tau = 1/sqrt(D),
+ *
+ * as named in "Fold-CP: A Context Parallelism Framework for Biomolecular
+ * Modeling" (Table 1, rows "Attn Pair Bias (Ring)" and "Triangle Attention";
+ * Figure 2 (a) and (c)).  The ring schemes there visit the keys block by
+ * block; each block yields an online-softmax partial (O, m, l) and a
+ * "tiled-softmax merge" combines them (the method of "Online normalizer
+ * calculation for softmax" and "Self-attention Does Not Need O(n2) Memory",
+ * both listed under "Builds on" on the page "Design-CP: Context Parallelism
+ * for Design of Protein Nanoparticles").  On one GPU the ring's P steps are P
+ * key blocks: pba_partial computes one block, softmax_merge combines them and
+ * pba_forward does the whole pass at once.
+ *
+ * Conventions common to every entry point
+ *   - Pointers marked "device" must be CUDA device memory of the current
+ *     device; the caller owns every buffer.  Per call the library allocates
+ *     nothing: it keeps one device error word and builds TMA descriptors on the
+ *     host stack.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Calls are thread-safe and keep no state
+ *     between calls apart from the error word.
+ *   - Natural logarithms throughout: lse = m + ln l, m = max of the scores.
+ *   - A key takes part if its mask byte is nonzero and its bias is not -inf.
+ *     A query row with no such key gets O = 0, lse = -inf (and m = -inf,
+ *     l = 0 for partials); never NaN.  Values of K and V must be finite,
+ *     masked keys included.  NaN or +inf in the inputs is outside the
+ *     contract.
+ *   - Return values: PBA_OK when the launch was enqueued.  PBA_ERR_INVALID_ARG
+ *     for a NULL required pointer, a negative size, a misaligned pointer or
+ *     stride (see below), or a size beyond the limits.  PBA_ERR_UNSUPPORTED for
+ *     a head dimension or dtype without a kernel, or a device that is not
+ *     sm_100.  PBA_ERR_CUDA when a CUDA runtime/driver call failed (the CUDA
+ *     error is left for cudaGetLastError).  Nothing is thrown across the ABI.
+ *   - Device-side faults are reported through pba_last_device_error(): every
+ *     wait inside the kernels is bounded (pba_set_wait_timeout_ns); a wait that
+ *     runs out records PBA_ERR_TIMEOUT and the kernel returns instead of
+ *     hanging.
+ *
+ * Alignment rules of the bf16 path (its tiles are moved by the Tensor Memory
+ * Accelerator): q, k, v and bias base addresses 16-byte aligned; every
+ * non-unit stride of q, k, v and bias a multiple of 8 elements (16 bytes).
+ * The bias row length may be ragged, but its row stride must be padded to a
+ * multiple of 8 elements.  For pba_partial the caller points k, v, bias and
+ * key_mask at the block's first key, so the block start must keep those rules
+ * (a multiple of 8 keys).  The fp32 path has no alignment rule beyond natural
+ * float alignment.
+ */
+#ifndef PBA_H
+#define PBA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported from libpba.so (the library is built with hidden visibility). */
+#if defined(__GNUC__)
+#define PBA_API __attribute__((visibility("default")))
+#else
+#define PBA_API
+#endif
+
+typedef enum {
+  PBA_OK = 0,
+  PBA_ERR_INVALID_ARG = 1,
+  PBA_ERR_UNSUPPORTED = 2,
+  PBA_ERR_CUDA = 3,
+  PBA_ERR_TIMEOUT = 4
+} pba_status;
+
+typedef enum { PBA_BF16 = 0, PBA_F32 = 1 } pba_dtype;
+
+typedef enum { PBA_TRI_STARTING = 0, PBA_TRI_ENDING = 1 } pba_tri_orient;
+
+/*
+ * Shape and layout of one pair-biased attention problem.
+ *   B, H       batch and heads (B, H >= 1)
+ *   Nq, Nk     query rows and keys (>= 0; Nk = 0 makes every row empty)
+ *   D          head dimension: 32 or 64 (bf16 and fp32)
+ *   dtype      pba_dtype of q, k, v, bias and of pba_forward's `out`
+ *   softmax_scale  tau; 0 selects 1/sqrt(D).  The bias is added unscaled.
+ *   *_stride   strides in ELEMENTS of the (b, h, n) axes; the d axis (and
+ *              the key axis of the bias) has stride 1.
+ *   bias_stride    (b, h, query row); a 0 in b or h broadcasts the bias over
+ *              that axis.
+ *   mask_stride_b  row stride of key_mask [B][Nk] (uint8, key stride 1).
+ *   out_stride     (b, h, n) of `out` / `o_part`, d stride 1.
+ *   lse_stride     (b, h, n) of `lse` / `m_part` / `l_part`.
+ */
+typedef struct {
+  int64_t B, H, Nq, Nk, D;
+  int32_t dtype;
+  float softmax_scale;
+  int64_t q_stride[3];
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t bias_stride[3];
+  int64_t mask_stride_b;
+  int64_t out_stride[3];
+  int64_t lse_stride[3];
+} pba_attn_desc;
+
+/*
+ * pba_forward -- one full pass over all Nk keys (Fold-CP, Table 1 "Attn
+ * Pair Bias"; the definition above).
+ *   q [B,H,Nq,D], k/v [B,H,Nk,D], bias [B,H,Nq,Nk]   device, desc->dtype
+ *   key_mask [B,Nk] uint8, device, or NULL (every key takes part)
+ *   out [B,H,Nq,D] device, desc->dtype: O (normalised)
+ *   lse [B,H,Nq] float, device, or NULL
+ */
+PBA_API pba_status pba_forward(const pba_attn_desc *desc, const void *q, const void *k, const void *v,
+                       const void *bias, const uint8_t *key_mask, void *out, float *lse, void *stream);
+
+/*
+ * pba_partial -- one ring step (Fold-CP, Figure 2(c): local queries against
+ * the key/value/bias block held): the online-softmax partial over the
+ * desc->Nk keys that k, v, bias and key_mask point at.
+ *   o_part [B,H,Nq,D] float: the block's output normalised by its own l
+ *   m_part [B,H,Nq] float: maximum score in the block (natural units)
+ *   l_part [B,H,Nq] float: sum over the block of exp(s - m_part)
+ * A block with no valid key for a row gives exactly (0, -inf, 0) there.
+ * bias_stride[2] is the row stride of the full bias matrix, so a block is a
+ * column window of it.
+ */
+PBA_API pba_status pba_partial(const pba_attn_desc *desc, const void *q, const void *k, const void *v,
+                       const void *bias, const uint8_t *key_mask, float *o_part, float *m_part, float *l_part,
+                       void *stream);
+
+/*
+ * softmax_merge -- the tiled-softmax merge (Fold-CP, Figure 2 (a) and (c)).
+ * P partials over disjoint key blocks, stacked in any order:
+ *   o_parts [P][rows][D], m_parts [P][rows], l_parts [P][rows]  float, device
+ * give, per row, M = max m_p over blocks with l_p > 0, w_p = l_p exp(m_p - M),
+ *   out = sum_p w_p o_p / sum_p w_p        [rows][D], out_dtype (bf16 or fp32)
+ *   lse = M + ln sum_p w_p                 [rows] float, or NULL
+ * A row with no valid key in any block gives out = 0, lse = -inf.
+ * P >= 1, rows >= 0, D a multiple of 4 up to 256; o_parts and out 16-byte
+ * aligned.
+ */
+PBA_API pba_status softmax_merge(int32_t P, int64_t rows, int64_t D, const float *o_parts, const float *m_parts,
+                         const float *l_parts, int32_t out_dtype, void *out, float *lse, void *stream);
+
+/*
+ * tri_attn_forward -- triangle attention on a pair tensor (Fold-CP, Table 1
+ * "Triangle Attention"; Figure 2(a)), bf16, heads H, head dim D in {32, 64}.
+ *   q, k, v, gate [N][N][H][D] (pair (i,j), then head, then d)  bf16, device
+ *   bias [H][N][N] bf16, device: the triangular bias, shared by all rows
+ *   pair_mask [N][N] uint8, device, or NULL
+ * Starting node (orient = PBA_TRI_STARTING), for every pair (i, j), head h:
+ *   o[i][j] = sum_k softmax_k( tau q[i][j].k[i][k] + b[h][j][k] ) v[i][k]
+ *   over keys k with pair_mask[i][k] != 0.
+ * Ending node (orient = PBA_TRI_ENDING):
+ *   o[i][j] = sum_k softmax_k( tau q[i][j].k[k][j] + b[h][k][i] ) v[k][j]
+ *   over keys k with pair_mask[k][j] != 0 -- the cross-axis transpose of
+ *   Figure 2(a), done by the tile loads' strides, not by a copy.
+ * out [N][N][H][D] bf16 = o * sigmoid(gate) (gate NULL: out = o);
+ * lse [N][N][H] float or NULL.  softmax_scale 0 selects 1/sqrt(D).
+ * N*H*D*2 bytes and H*D*2 bytes are the tile strides, so H*D must be a
+ * multiple of 8 and N a multiple of 8.
+ */
+PBA_API pba_status tri_attn_forward(int64_t N, int64_t H, int64_t D, int32_t orient, float softmax_scale, const void *q,
+                            const void *k, const void *v, const void *bias, const void *gate,
+                            const uint8_t *pair_mask, void *out, float *lse, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+PBA_API const char *pba_status_string(pba_status status);
+
+/*
+ * pba_last_device_error -- synchronises `stream`, then returns and clears the
+ * device error word of the current device (PBA_OK if no kernel recorded an
+ * error since the last call; PBA_ERR_TIMEOUT if a bounded wait ran out).
+ * Returns PBA_ERR_CUDA if the synchronisation itself failed.
+ */
+PBA_API pba_status pba_last_device_error(void *stream);
+
+/*
+ * pba_set_wait_timeout_ns -- limit of every wait inside the kernels, in
+ * nanoseconds of GPU global time (default 1e9 = 1 s; 0 restores the default).
+ * Applies to launches made after the call.  Returns the previous value.
+ */
+PBA_API uint64_t pba_set_wait_timeout_ns(uint64_t timeout_ns);
+
+/*
+ * pba_selftest_wait_timeout -- launches one block that waits on a barrier
+ * that nothing will ever complete, with a wait limit of `timeout_ns`, so that
+ * the bounded-wait path can be checked without hanging the GPU.  The kernel
+ * records PBA_ERR_TIMEOUT in the device error word and returns; read it with
+ * pba_last_device_error.  No counterpart on the pages: it tests this
+ * library's failure detection.
+ */
+PBA_API pba_status pba_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PBA_H */

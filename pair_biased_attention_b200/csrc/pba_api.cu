@@ -1,0 +1,477 @@
+// pba_api.cu -- the C ABI declared in include/pba.h: argument checks, Tensor
+// Memory Accelerator descriptors and kernel launches.  Every step of the
+// computation runs in the kernels of pba_attn_sm100.cuh and pba_simt.cuh.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "pba.h"
+#include "pba_attn_sm100.cuh"
+#include "pba_simt.cuh"
+
+// Device error word: written by kernels whose bounded waits ran out, read and
+// cleared by pba_last_device_error().
+__device__ int g_pba_err = 0;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
+std::atomic<uint64_t> g_timeout_ns{kDefaultTimeoutNs};
+
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+pba_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PBA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return PBA_ERR_CUDA;
+  if (major != 10 || minor != 0) return PBA_ERR_UNSUPPORTED;  // built for sm_100a only
+  return PBA_OK;
+}
+
+int *device_error_word() {
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_pba_err) != cudaSuccess) return nullptr;
+  return static_cast<int *>(p);
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kMaxI32 = 2147483647;
+
+// 4-D tiled tensor map of bf16 elements.  dims/strides innermost first;
+// strides in bytes for dims 1..3.  A dim of extent 1 gets a harmless positive
+// stride (its coordinate is always 0).
+bool make_map(CUtensorMap *map, const void *base, const uint64_t dims[4], const int64_t strides_bytes[3],
+              const uint32_t box[4], CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t gdim[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gstride[3];
+  int64_t prev_extent = int64_t(dims[0]) * 2;
+  for (int i = 0; i < 3; ++i) {
+    int64_t s = strides_bytes[i];
+    if (dims[i + 1] == 1 || s <= 0) s = (prev_extent + 15) / 16 * 16;
+    gstride[i] = cuuint64_t(s);
+    prev_extent = s * int64_t(dims[i + 1]);
+  }
+  cuuint32_t bdim[4] = {box[0], box[1], box[2], box[3]};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), gdim, gstride, bdim, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool stride_ok_bf16(int64_t s, int64_t extent) { return extent <= 1 || (s > 0 && s % 8 == 0); }
+
+// ------------------------------------------------------------ tensor-core path
+struct TcProblem {
+  int B, H, Nq, Nk, D;
+  float tau;
+  const void *q, *k, *v, *bias;
+  int64_t q_s[3], k_s[3], v_s[3];  // (b, h, n) elements
+  // bias: either [query][key] rows (bias_t = false) or [key][query] rows (true)
+  bool bias_t;
+  int64_t bias_s[3];  // (b, h, row) elements
+  bool bias_b_bcast, bias_h_bcast;
+  const uint8_t *mask;
+  int64_t mask_sb, mask_sk;
+  int epi;  // pba::kEpiForward / kEpiPartial
+  void *out;
+  int64_t out_s[3];
+  float *lse;
+  int64_t lse_s[3];
+  float *l_part;
+  const void *gate;
+  int64_t gate_s[3];
+};
+
+template <int D, bool kBiasT, int kEpi, bool kGate>
+cudaError_t launch_tc(const pba::AttnParams &p, int grid, cudaStream_t stream) {
+  using L = pba::AttnLayout<D>;
+  auto kern = pba::pba_attn_sm100_kernel<D, kBiasT, kEpi, kGate>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, pba::kAttnThreads, L::kSmemAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_tc(const pba::AttnParams &p, int grid, bool bias_t, int epi, bool gate, cudaStream_t st) {
+  if (epi == pba::kEpiPartial) return launch_tc<D, false, pba::kEpiPartial, false>(p, grid, st);
+  if (!bias_t && !gate) return launch_tc<D, false, pba::kEpiForward, false>(p, grid, st);
+  if (!bias_t && gate) return launch_tc<D, false, pba::kEpiForward, true>(p, grid, st);
+  if (bias_t && !gate) return launch_tc<D, true, pba::kEpiForward, false>(p, grid, st);
+  return launch_tc<D, true, pba::kEpiForward, true>(p, grid, st);
+}
+
+pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
+  pba::AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint32_t qbox[4] = {uint32_t(t.D), uint32_t(pba::kBM), 1, 1};
+  const uint32_t kbox[4] = {uint32_t(t.D), uint32_t(pba::kBN), 1, 1};
+  const CUtensorMapSwizzle swz = (t.D == 64) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  {
+    const uint64_t dims[4] = {uint64_t(t.D), uint64_t(t.Nq), uint64_t(t.H), uint64_t(t.B)};
+    const int64_t st[3] = {t.q_s[2] * 2, t.q_s[1] * 2, t.q_s[0] * 2};
+    if (!make_map(&p.tm_q, t.q, dims, st, qbox, swz)) return PBA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(t.D), uint64_t(t.Nk), uint64_t(t.H), uint64_t(t.B)};
+    const int64_t sk[3] = {t.k_s[2] * 2, t.k_s[1] * 2, t.k_s[0] * 2};
+    const int64_t sv[3] = {t.v_s[2] * 2, t.v_s[1] * 2, t.v_s[0] * 2};
+    if (!make_map(&p.tm_k, t.k, dims, sk, kbox, swz)) return PBA_ERR_INVALID_ARG;
+    if (!make_map(&p.tm_v, t.v, dims, sv, kbox, swz)) return PBA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t hb = t.bias_h_bcast ? 1 : uint64_t(t.H), bb = t.bias_b_bcast ? 1 : uint64_t(t.B);
+    const int64_t st[3] = {t.bias_s[2] * 2, t.bias_s[1] * 2, t.bias_s[0] * 2};
+    if (t.bias_t) {
+      const uint64_t dims[4] = {uint64_t(t.Nq), uint64_t(t.Nk), hb, bb};
+      const uint32_t box[4] = {uint32_t(pba::kBM), uint32_t(pba::kBN), 1, 1};
+      if (!make_map(&p.tm_bias, t.bias, dims, st, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return PBA_ERR_INVALID_ARG;
+    } else {
+      const uint64_t dims[4] = {uint64_t(t.Nk), uint64_t(t.Nq), hb, bb};
+      const uint32_t box[4] = {64, uint32_t(pba::kBM), 1, 1};
+      if (!make_map(&p.tm_bias, t.bias, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+    }
+  }
+  p.B = t.B;
+  p.H = t.H;
+  p.Nq = t.Nq;
+  p.Nk = t.Nk;
+  p.n_qblocks = (t.Nq + pba::kQTiles * pba::kBM - 1) / (pba::kQTiles * pba::kBM);
+  p.bias_h_bcast = t.bias_h_bcast;
+  p.bias_b_bcast = t.bias_b_bcast;
+  p.needs_mask = (t.mask != nullptr) || (t.Nk % pba::kBN != 0);
+  p.tau = t.tau;
+  p.mask = t.mask;
+  p.mask_sb = t.mask_sb;
+  p.mask_sk = t.mask_sk;
+  p.out = t.out;
+  p.out_sb = t.out_s[0];
+  p.out_sh = t.out_s[1];
+  p.out_sn = t.out_s[2];
+  p.lse = t.lse;
+  p.lse_sb = t.lse_s[0];
+  p.lse_sh = t.lse_s[1];
+  p.lse_sn = t.lse_s[2];
+  p.l_part = t.l_part;
+  p.gate = static_cast<const uint16_t *>(t.gate);
+  p.gate_sb = t.gate_s[0];
+  p.gate_sh = t.gate_s[1];
+  p.gate_sn = t.gate_s[2];
+  p.err = device_error_word();
+  if (p.err == nullptr) return PBA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
+  const int64_t grid = int64_t(t.B) * t.H * p.n_qblocks;
+  if (grid > kMaxI32) return PBA_ERR_INVALID_ARG;
+  cudaError_t e = (t.D == 64) ? dispatch_tc<64>(p, int(grid), t.bias_t, t.epi, t.gate != nullptr, stream)
+                              : dispatch_tc<32>(p, int(grid), t.bias_t, t.epi, t.gate != nullptr, stream);
+  return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------ shared checks
+pba_status check_desc(const pba_attn_desc *d) {
+  if (d == nullptr) return PBA_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->Nq < 0 || d->Nk < 0) return PBA_ERR_INVALID_ARG;
+  if (d->B > kMaxI32 || d->H > kMaxI32 || d->Nq > kMaxI32 || d->Nk > kMaxI32) return PBA_ERR_INVALID_ARG;
+  if (d->dtype != PBA_BF16 && d->dtype != PBA_F32) return PBA_ERR_UNSUPPORTED;
+  if (d->D != 32 && d->D != 64) return PBA_ERR_UNSUPPORTED;
+  if (!(d->softmax_scale >= 0.f) || std::isinf(d->softmax_scale)) return PBA_ERR_INVALID_ARG;
+  return PBA_OK;
+}
+
+float tau_of(float scale, int64_t D) { return scale > 0.f ? scale : float(1.0 / std::sqrt(double(D))); }
+
+pba_status launch_empty(const pba_attn_desc *d, bool partial, void *out, float *lse, float *l_part,
+                        cudaStream_t stream) {
+  pba::EmptyParams e;
+  e.B = int(d->B);
+  e.H = int(d->H);
+  e.Nq = int(d->Nq);
+  e.D = int(d->D);
+  e.out_bf16 = (!partial && d->dtype == PBA_BF16) ? 1 : 0;
+  e.partial = partial ? 1 : 0;
+  e.out = out;
+  e.out_sb = d->out_stride[0];
+  e.out_sh = d->out_stride[1];
+  e.out_sn = d->out_stride[2];
+  e.lse = lse;
+  e.lse_sb = d->lse_stride[0];
+  e.lse_sh = d->lse_stride[1];
+  e.lse_sn = d->lse_stride[2];
+  e.l_part = l_part;
+  pba::pba_empty_keys_kernel<<<296, 256, 0, stream>>>(e);
+  return cudaGetLastError() == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+pba_status attn_common(const pba_attn_desc *d, const void *q, const void *k, const void *v, const void *bias,
+                       const uint8_t *mask, bool partial, void *out, float *lse, float *l_part, void *stream_ptr) {
+  pba_status s = check_desc(d);
+  if (s != PBA_OK) return s;
+  if (q == nullptr || k == nullptr || v == nullptr || bias == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
+  if (partial && (lse == nullptr || l_part == nullptr)) return PBA_ERR_INVALID_ARG;
+  s = check_device();
+  if (s != PBA_OK) return s;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (d->Nq == 0) return PBA_OK;
+  if (d->Nk == 0) return launch_empty(d, partial, out, lse, l_part, stream);
+  const float tau = tau_of(d->softmax_scale, d->D);
+
+  if (d->dtype == PBA_F32) {
+    pba::SimtParams p;
+    p.B = int(d->B);
+    p.H = int(d->H);
+    p.Nq = int(d->Nq);
+    p.Nk = int(d->Nk);
+    p.tau = tau;
+    p.q = static_cast<const float *>(q);
+    p.k = static_cast<const float *>(k);
+    p.v = static_cast<const float *>(v);
+    p.bias = static_cast<const float *>(bias);
+    p.q_sb = d->q_stride[0], p.q_sh = d->q_stride[1], p.q_sn = d->q_stride[2];
+    p.k_sb = d->k_stride[0], p.k_sh = d->k_stride[1], p.k_sn = d->k_stride[2];
+    p.v_sb = d->v_stride[0], p.v_sh = d->v_stride[1], p.v_sn = d->v_stride[2];
+    p.bias_sb = d->bias_stride[0], p.bias_sh = d->bias_stride[1], p.bias_sn = d->bias_stride[2];
+    p.mask = mask;
+    p.mask_sb = d->mask_stride_b;
+    p.out = static_cast<float *>(out);
+    p.out_sb = d->out_stride[0], p.out_sh = d->out_stride[1], p.out_sn = d->out_stride[2];
+    p.lse = lse;
+    p.lse_sb = d->lse_stride[0], p.lse_sh = d->lse_stride[1], p.lse_sn = d->lse_stride[2];
+    p.l_part = l_part;
+    const int64_t rows = d->B * d->H * d->Nq;
+    const int64_t grid = (rows + 3) / 4;
+    if (grid > kMaxI32) return PBA_ERR_INVALID_ARG;
+    if (d->D == 64) {
+      if (partial)
+        pba::pba_attn_f32_kernel<64, true><<<int(grid), 128, 0, stream>>>(p);
+      else
+        pba::pba_attn_f32_kernel<64, false><<<int(grid), 128, 0, stream>>>(p);
+    } else {
+      if (partial)
+        pba::pba_attn_f32_kernel<32, true><<<int(grid), 128, 0, stream>>>(p);
+      else
+        pba::pba_attn_f32_kernel<32, false><<<int(grid), 128, 0, stream>>>(p);
+    }
+    return cudaGetLastError() == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+  }
+
+  // bf16 on the tensor cores: tile loads need 16-byte aligned bases and strides
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) || !aligned16(out))
+    return PBA_ERR_INVALID_ARG;
+  const int64_t *qs = d->q_stride, *ks = d->k_stride, *vs = d->v_stride, *bs = d->bias_stride;
+  if (!stride_ok_bf16(qs[0], d->B) || !stride_ok_bf16(qs[1], d->H) || !stride_ok_bf16(qs[2], d->Nq) ||
+      !stride_ok_bf16(ks[0], d->B) || !stride_ok_bf16(ks[1], d->H) || !stride_ok_bf16(ks[2], d->Nk) ||
+      !stride_ok_bf16(vs[0], d->B) || !stride_ok_bf16(vs[1], d->H) || !stride_ok_bf16(vs[2], d->Nk) ||
+      !stride_ok_bf16(bs[2], d->Nq))
+    return PBA_ERR_INVALID_ARG;
+  if ((bs[0] != 0 && !stride_ok_bf16(bs[0], d->B)) || (bs[1] != 0 && !stride_ok_bf16(bs[1], d->H)))
+    return PBA_ERR_INVALID_ARG;
+  // outputs: 16-byte vector stores of whole rows
+  const int64_t out_mult = partial ? 4 : 8;
+  for (int i = 0; i < 3; ++i)
+    if (d->out_stride[i] % out_mult != 0) return PBA_ERR_INVALID_ARG;
+  TcProblem t;
+  std::memset(&t, 0, sizeof(t));
+  t.B = int(d->B);
+  t.H = int(d->H);
+  t.Nq = int(d->Nq);
+  t.Nk = int(d->Nk);
+  t.D = int(d->D);
+  t.tau = tau;
+  t.q = q;
+  t.k = k;
+  t.v = v;
+  t.bias = bias;
+  for (int i = 0; i < 3; ++i) {
+    t.q_s[i] = qs[i];
+    t.k_s[i] = ks[i];
+    t.v_s[i] = vs[i];
+    t.bias_s[i] = bs[i];
+    t.out_s[i] = d->out_stride[i];
+    t.lse_s[i] = d->lse_stride[i];
+  }
+  t.bias_t = false;
+  t.bias_b_bcast = bs[0] == 0;
+  t.bias_h_bcast = bs[1] == 0;
+  t.mask = mask;
+  t.mask_sb = d->mask_stride_b;
+  t.mask_sk = 1;
+  t.epi = partial ? pba::kEpiPartial : pba::kEpiForward;
+  t.out = out;
+  t.lse = lse;
+  t.l_part = l_part;
+  t.gate = nullptr;
+  return run_tc(t, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+pba_status pba_forward(const pba_attn_desc *desc, const void *q, const void *k, const void *v, const void *bias,
+                       const uint8_t *key_mask, void *out, float *lse, void *stream) {
+  return attn_common(desc, q, k, v, bias, key_mask, false, out, lse, nullptr, stream);
+}
+
+pba_status pba_partial(const pba_attn_desc *desc, const void *q, const void *k, const void *v, const void *bias,
+                       const uint8_t *key_mask, float *o_part, float *m_part, float *l_part, void *stream) {
+  return attn_common(desc, q, k, v, bias, key_mask, true, o_part, m_part, l_part, stream);
+}
+
+pba_status softmax_merge(int32_t P, int64_t rows, int64_t D, const float *o_parts, const float *m_parts,
+                         const float *l_parts, int32_t out_dtype, void *out, float *lse, void *stream_ptr) {
+  if (P < 1 || rows < 0 || D < 4 || D > 256 || D % 4 != 0) return PBA_ERR_INVALID_ARG;
+  if (out_dtype != PBA_BF16 && out_dtype != PBA_F32) return PBA_ERR_UNSUPPORTED;
+  if (o_parts == nullptr || m_parts == nullptr || l_parts == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || (reinterpret_cast<uintptr_t>(out) & (out_dtype == PBA_BF16 ? 7u : 15u)) != 0)
+    return PBA_ERR_INVALID_ARG;
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  if (rows == 0) return PBA_OK;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t total = rows * (D / 4);
+  int64_t grid = (total + 255) / 256;
+  const int64_t cap = int64_t(sms) * 8;  // a few resident blocks per SM, grid-stride beyond
+  if (grid > cap) grid = cap;
+  if (out_dtype == PBA_BF16)
+    pba::softmax_merge_kernel<true><<<int(grid), 256, 0, stream>>>(P, rows, int(D), o_parts, m_parts, l_parts, out,
+                                                                    lse);
+  else
+    pba::softmax_merge_kernel<false><<<int(grid), 256, 0, stream>>>(P, rows, int(D), o_parts, m_parts, l_parts,
+                                                                     out, lse);
+  return cudaGetLastError() == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+pba_status tri_attn_forward(int64_t N, int64_t H, int64_t D, int32_t orient, float softmax_scale, const void *q,
+                            const void *k, const void *v, const void *bias, const void *gate,
+                            const uint8_t *pair_mask, void *out, float *lse, void *stream_ptr) {
+  if (N < 0 || H < 1 || N > 65535 || H > 4096) return PBA_ERR_INVALID_ARG;
+  if (D != 32 && D != 64) return PBA_ERR_UNSUPPORTED;
+  if (orient != PBA_TRI_STARTING && orient != PBA_TRI_ENDING) return PBA_ERR_INVALID_ARG;
+  if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return PBA_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || bias == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) || !aligned16(out) ||
+      (gate != nullptr && !aligned16(gate)))
+    return PBA_ERR_INVALID_ARG;
+  if (N % 8 != 0 || (H * D) % 8 != 0) return PBA_ERR_INVALID_ARG;
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  if (N == 0) return PBA_OK;
+  const bool ending = orient == PBA_TRI_ENDING;
+  const int64_t HD = H * D, NHD = N * H * D;
+  TcProblem t;
+  std::memset(&t, 0, sizeof(t));
+  t.B = int(N);  // one problem per pair-tensor line
+  t.H = int(H);
+  t.Nq = int(N);
+  t.Nk = int(N);
+  t.D = int(D);
+  t.tau = tau_of(softmax_scale, D);
+  t.q = q;
+  t.k = k;
+  t.v = v;
+  t.bias = bias;
+  // (line, head, position): starting node line = row i, position = column j;
+  // ending node line = column j, position = row i (outer strides swapped).
+  const int64_t s_line = ending ? HD : NHD, s_pos = ending ? NHD : HD;
+  const int64_t qkv_s[3] = {s_line, D, s_pos};
+  for (int i = 0; i < 3; ++i) {
+    t.q_s[i] = qkv_s[i];
+    t.k_s[i] = qkv_s[i];
+    t.v_s[i] = qkv_s[i];
+    t.out_s[i] = qkv_s[i];
+    t.gate_s[i] = qkv_s[i];
+  }
+  // bias [H][N][N]: starting node reads rows b[h][j][:] (query j, keys k);
+  // ending node reads b[h][k][i] as a [key][query] tile.
+  t.bias_t = ending;
+  t.bias_s[0] = 0;
+  t.bias_s[1] = N * N;
+  t.bias_s[2] = N;
+  t.bias_b_bcast = true;
+  t.bias_h_bcast = false;
+  t.mask = pair_mask;
+  t.mask_sb = ending ? 1 : N;
+  t.mask_sk = ending ? N : 1;
+  t.epi = pba::kEpiForward;
+  t.out = out;
+  t.lse = lse;
+  t.lse_s[0] = ending ? H : N * H;
+  t.lse_s[1] = 1;
+  t.lse_s[2] = ending ? N * H : H;
+  t.gate = gate;
+  return run_tc(t, static_cast<cudaStream_t>(stream_ptr));
+}
+
+const char *pba_status_string(pba_status status) {
+  switch (status) {
+    case PBA_OK:
+      return "PBA_OK";
+    case PBA_ERR_INVALID_ARG:
+      return "PBA_ERR_INVALID_ARG";
+    case PBA_ERR_UNSUPPORTED:
+      return "PBA_ERR_UNSUPPORTED";
+    case PBA_ERR_CUDA:
+      return "PBA_ERR_CUDA";
+    case PBA_ERR_TIMEOUT:
+      return "PBA_ERR_TIMEOUT";
+  }
+  return "PBA_ERR_UNKNOWN";
+}
+
+pba_status pba_last_device_error(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PBA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_pba_err, sizeof(int)) != cudaSuccess) return PBA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_pba_err, &zero, sizeof(int)) != cudaSuccess) return PBA_ERR_CUDA;
+  }
+  return static_cast<pba_status>(v);
+}
+
+uint64_t pba_set_wait_timeout_ns(uint64_t timeout_ns) {
+  return g_timeout_ns.exchange(timeout_ns == 0 ? kDefaultTimeoutNs : timeout_ns);
+}
+
+pba_status pba_selftest_wait_timeout(uint64_t timeout_ns, void *stream) {
+  if (timeout_ns == 0 || timeout_ns > 10ull * kDefaultTimeoutNs) return PBA_ERR_INVALID_ARG;
+  int *err = device_error_word();
+  if (err == nullptr) return PBA_ERR_CUDA;
+  pba::pba_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,519 @@
+// pba_attn_sm100.cuh -- pair-biased attention on the sm_100a tensor cores.
+//
+// Computes, per (batch b, head h) and query row i,
+//     O_i = sum_j softmax_j( tau q_i.k_j + b_ij ) v_j
+// over the key tiles of one call, as in "Fold-CP: A Context Parallelism
+// Framework for Biomolecular Modeling" (Table 1 "Attn Pair Bias", Figure 2(c):
+// attention of the local queries against a key/value/pair-bias block).  The
+// softmax is accumulated online, tile by tile (the method of "Online
+// normalizer calculation for softmax", listed under "Builds on" on the
+// "Design-CP" page), so the same main loop serves a full pass (epilogue:
+// bf16 O and the log-sum-exp) and one ring step (epilogue: the fp32 partial
+// O_p, m_p, l_p that the tiled-softmax merge combines).  Triangle attention
+// runs the same loop with the pair-tensor strides in the tile descriptors.
+//
+// One CTA per SM holds two 128-row query tiles of one (b, h):
+//   warps 0-3   softmax warpgroup for query tile 0 (thread t owns row t)
+//   warps 4-7   softmax warpgroup for query tile 1
+//   warp 8      TMA producer: Q once, then K, V and the two bias tiles per
+//               128-key tile, through shared-memory rings
+//   warp 9      allocates Tensor Memory and issues every tcgen05.mma
+//   warp 10     key-mask warp: writes -inf into the bias tile columns of
+//               masked keys and of keys past the end, in shared memory, before
+//               the softmax warps read the tile
+// Tensor Memory (512 columns x 128 lanes of fp32):
+//   [0,128) S0   [128,256) S1   [256,320) P0   [320,384) P1
+//   [384,384+D) O0   [448,448+D) O1
+// S_w = Q_w K^T (fp32), P_w = bf16 probabilities (two per column), O_w the
+// running output.  The MMA warp issues S0(j), PV0(j-1), S1(j), PV1(j-1), so
+// the next score tile is computed while the softmax warps work on this one.
+#pragma once
+
+#include <cuda.h>
+
+#include "pba_ptx.cuh"
+
+namespace pba {
+
+constexpr int kBM = 128;          // query rows per tile (one TMEM lane each)
+constexpr int kBN = 128;          // keys per tile
+constexpr int kQTiles = 2;        // query tiles per CTA
+constexpr int kBiasStages = 2;    // bias ring depth per softmax warpgroup
+constexpr int kAttnThreads = 352; // 11 warps
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr int kWarpMask = 10;
+constexpr uint32_t kTmemCols = 512;
+
+enum Epilogue : int { kEpiForward = 0, kEpiPartial = 1 };
+
+struct AttnParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_bias;
+  int32_t B, H, Nq, Nk;
+  int32_t n_qblocks;     // ceil(Nq / 256)
+  int32_t bias_h_bcast;  // bias head stride 0
+  int32_t bias_b_bcast;  // bias batch stride 0
+  int32_t needs_mask;    // key mask given or Nk not a multiple of the key tile
+  float tau;
+  const uint8_t *mask;
+  int64_t mask_sb, mask_sk;
+  void *out;  // bf16 O (forward) or fp32 O_p (partial)
+  int64_t out_sb, out_sh, out_sn;
+  float *lse;  // forward: log-sum-exp; partial: m_p
+  int64_t lse_sb, lse_sh, lse_sn;
+  float *l_part;  // partial: l_p (strides of lse)
+  const uint16_t *gate;
+  int64_t gate_sb, gate_sh, gate_sn;
+  int *err;
+  uint64_t timeout_ns;
+};
+
+template <int D>
+struct AttnLayout {
+  static_assert(D == 32 || D == 64, "head dimension");
+  static constexpr int kRowBytes = D * 2;                   // one bf16 row of Q/K/V
+  static constexpr int kSwizzleMode = (D == 64) ? 2 : 4;    // 128-byte / 64-byte swizzle
+  static constexpr int kAtomBytes = 8 * kRowBytes;          // 8-row swizzle atom
+  static constexpr int kKVStages = (D == 64) ? 2 : 4;
+  static constexpr int kQBytes = kBM * kRowBytes;
+  static constexpr int kKVBytes = kBN * kRowBytes;
+  static constexpr int kBiasBytes = kBM * kBN * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQTiles * kQBytes;
+  static constexpr int kOffV = kOffK + kKVStages * kKVBytes;
+  static constexpr int kOffBias = kOffV + kKVStages * kKVBytes;
+  static constexpr int kOffBar = kOffBias + kQTiles * kBiasStages * kBiasBytes;
+  // barriers
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarKFull = 1;
+  static constexpr int kBarVFull = kBarKFull + kKVStages;
+  static constexpr int kBarKVEmpty = kBarVFull + kKVStages;
+  static constexpr int kBarBiasFull = kBarKVEmpty + kKVStages;            // [w][t]
+  static constexpr int kBarBiasReady = kBarBiasFull + kQTiles * kBiasStages;
+  static constexpr int kBarBiasEmpty = kBarBiasReady + kQTiles * kBiasStages;
+  static constexpr int kBarSFull = kBarBiasEmpty + kQTiles * kBiasStages;  // [w]
+  static constexpr int kBarSFree = kBarSFull + kQTiles;
+  static constexpr int kBarPFull = kBarSFree + kQTiles;
+  static constexpr int kBarODone = kBarPFull + kQTiles;
+  static constexpr int kBarDrain = kBarODone + kQTiles;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemSlot + 4;
+  static constexpr int kBytes = kOffAbort + 4;
+  static constexpr int kSmemAlloc = kBytes + 1024;  // room to align the base to 1024
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+};
+
+// Natural-log constants of the base-2 softmax.
+constexpr float kLog2e = 1.4426950408889634f;
+// A row keeps its running maximum until a tile's maximum exceeds it by more
+// than 8 (in log2 units), so most tiles skip the rescale of O; the stale
+// maximum is used consistently for P and l, so the result is unchanged and the
+// probabilities stay below 2^8.
+constexpr float kRescaleThreshold = 8.0f / kLog2e;
+
+template <int D, bool kBiasT, int kEpi, bool kGate>
+__global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const __grid_constant__ AttnParams p) {
+  using L = AttnLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmemSlot);
+  int *abort_flag = reinterpret_cast<int *>(smem + L::kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: (b, h, 256 query rows)
+  const int unit = blockIdx.x;
+  const int qblk = unit % p.n_qblocks;
+  const int bh = unit / p.n_qblocks;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
+  const int q0 = qblk * (kQTiles * kBM);
+  const int nt = (p.Nk + kBN - 1) / kBN;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[L::kBarQFull], 1);
+    for (int s = 0; s < L::kKVStages; ++s) {
+      mbar_init(&bars[L::kBarKFull + s], 1);
+      mbar_init(&bars[L::kBarVFull + s], 1);
+      mbar_init(&bars[L::kBarKVEmpty + s], 1);
+    }
+    for (int i = 0; i < kQTiles * kBiasStages; ++i) {
+      mbar_init(&bars[L::kBarBiasFull + i], 1);
+      mbar_init(&bars[L::kBarBiasReady + i], 32);
+      mbar_init(&bars[L::kBarBiasEmpty + i], kBM);
+    }
+    for (int w = 0; w < kQTiles; ++w) {
+      mbar_init(&bars[L::kBarSFull + w], 1);
+      mbar_init(&bars[L::kBarSFree + w], kBM);
+      mbar_init(&bars[L::kBarPFull + w], kBM);
+      mbar_init(&bars[L::kBarODone + w], 1);
+    }
+    mbar_init(&bars[L::kBarDrain], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    tma_prefetch_desc(&p.tm_bias);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.err, p.timeout_ns};
+  WaitCtl wc_drain = wc;  // clean-up waits: ignore the abort word, keep the time limit
+  int drain_abort = 0;
+  wc_drain.abort_flag = &drain_abort;
+
+  const int hb = p.bias_h_bcast ? 0 : h;
+  const int bb = p.bias_b_bcast ? 0 : b;
+
+  if (warp == kWarpProducer) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = l2_policy_evict_first();
+      const uint64_t pol_keep = l2_policy_evict_last();
+      bool ok = true;
+      // times each full barrier was armed, for the clean-up on abort
+      int arms_k[L::kKVStages] = {}, arms_v[L::kKVStages] = {}, arms_b[kQTiles * kBiasStages] = {};
+      mbar_arrive_expect_tx(&bars[L::kBarQFull], kQTiles * L::kQBytes);
+      for (int w = 0; w < kQTiles; ++w)
+        tma_load_4d(smem + L::kOffQ + w * L::kQBytes, &p.tm_q, &bars[L::kBarQFull], 0, q0 + w * kBM, h, b,
+                    pol_stream);
+      for (int j = 0; j < nt && ok; ++j) {
+        const int s = j % L::kKVStages;
+        if (j >= L::kKVStages) ok = mbar_wait(&bars[L::kBarKVEmpty + s], ((j / L::kKVStages) - 1) & 1, wc);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kKVBytes);
+        tma_load_4d(smem + L::kOffK + s * L::kKVBytes, &p.tm_k, &bars[L::kBarKFull + s], 0, j * kBN, h, b,
+                    pol_keep);
+        ++arms_k[s];
+        mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kKVBytes);
+        tma_load_4d(smem + L::kOffV + s * L::kKVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kBN, h, b,
+                    pol_keep);
+        ++arms_v[s];
+        const int t = j % kBiasStages;
+        for (int w = 0; w < kQTiles && ok; ++w) {
+          const int slot = w * kBiasStages + t;
+          if (j >= kBiasStages) ok = mbar_wait(&bars[L::kBarBiasEmpty + slot], ((j / kBiasStages) - 1) & 1, wc);
+          if (!ok) break;
+          uint8_t *dst = smem + L::kOffBias + slot * L::kBiasBytes;
+          mbar_arrive_expect_tx(&bars[L::kBarBiasFull + slot], L::kBiasBytes);
+          if (kBiasT) {
+            // transposed bias tile: [128 keys][128 queries], no swizzle
+            tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], q0 + w * kBM, j * kBN, hb, bb, pol_stream);
+          } else {
+            // [128 queries][128 keys] as two 64-key boxes, 128-byte swizzle
+            tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN, q0 + w * kBM, hb, bb, pol_stream);
+            tma_load_4d(dst + L::kBiasBytes / 2, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN + 64,
+                        q0 + w * kBM, hb, bb, pol_stream);
+          }
+          ++arms_b[slot];
+        }
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA exits: each full
+        // barrier has at most one armed phase that no consumer has waited for.
+        mbar_wait(&bars[L::kBarQFull], 0, wc_drain);
+        for (int s = 0; s < L::kKVStages; ++s) {
+          if (arms_k[s]) mbar_wait(&bars[L::kBarKFull + s], (arms_k[s] - 1) & 1, wc_drain);
+          if (arms_v[s]) mbar_wait(&bars[L::kBarVFull + s], (arms_v[s] - 1) & 1, wc_drain);
+        }
+        for (int i = 0; i < kQTiles * kBiasStages; ++i)
+          if (arms_b[i]) mbar_wait(&bars[L::kBarBiasFull + i], (arms_b[i] - 1) & 1, wc_drain);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);
+      const uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
+      const uint32_t sQ = smem_u32(smem + L::kOffQ);
+      const uint32_t sK = smem_u32(smem + L::kOffK);
+      const uint32_t sV = smem_u32(smem + L::kOffV);
+      bool ok = mbar_wait(&bars[L::kBarQFull], 0, wc);
+      auto issue_s = [&](int w, int j) {
+        const int s = j % L::kKVStages;
+        const uint32_t d_tmem = tmem + w * kBN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = smem_desc(sQ + w * L::kQBytes + kk * 32, 16, L::kAtomBytes, L::kSwizzleMode);
+          const uint64_t bdesc = smem_desc(sK + s * L::kKVBytes + kk * 32, 16, L::kAtomBytes, L::kSwizzleMode);
+          mma_bf16_ss(d_tmem, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[L::kBarSFull + w]);
+      };
+      auto issue_pv = [&](int w, int j) {
+        const int s = j % L::kKVStages;
+        const uint32_t d_tmem = tmem + 384 + w * 64;
+        const uint32_t a_tmem = tmem + 256 + w * 64;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bdesc = smem_desc(sV + s * L::kKVBytes + kk * 16 * L::kRowBytes, L::kKVBytes, L::kAtomBytes,
+                                           L::kSwizzleMode);
+          mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars[L::kBarODone + w]);
+      };
+      for (int j = 0; j < nt && ok; ++j) {
+        const int s = j % L::kKVStages;
+        ok = mbar_wait(&bars[L::kBarKFull + s], (j / L::kKVStages) & 1, wc);
+        for (int w = 0; w < kQTiles && ok; ++w) {
+          if (j > 0) ok = mbar_wait(&bars[L::kBarSFree + w], (j - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_s(w, j);
+          if (j > 0) {
+            const int sp = (j - 1) % L::kKVStages;
+            ok = mbar_wait(&bars[L::kBarPFull + w], (j - 1) & 1, wc) &&
+                 mbar_wait(&bars[L::kBarVFull + sp], ((j - 1) / L::kKVStages) & 1, wc);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_pv(w, j - 1);
+            if (w == kQTiles - 1) tc_commit(&bars[L::kBarKVEmpty + sp]);
+          }
+        }
+      }
+      for (int w = 0; w < kQTiles && ok; ++w) {
+        const int sp = (nt - 1) % L::kKVStages;
+        ok = mbar_wait(&bars[L::kBarPFull + w], (nt - 1) & 1, wc) &&
+             mbar_wait(&bars[L::kBarVFull + sp], ((nt - 1) / L::kKVStages) & 1, wc);
+        if (!ok) break;
+        tc_fence_after_sync();
+        issue_pv(w, nt - 1);
+      }
+      // Every MMA issued above completes before Tensor Memory is released.
+      tc_commit(&bars[L::kBarDrain]);
+      mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
+    }
+  } else if (warp == kWarpMask) {
+    // ================================================================ key-mask warp
+    // Without a key mask and with whole key tiles the softmax warps wait on
+    // the TMA barrier directly and this warp has nothing to do.
+    bool ok = p.needs_mask != 0;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int k0 = j * kBN;
+      uint32_t inv = 0;  // bit e: key k0 + 4*lane + e is masked or past the end
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = k0 + 4 * lane + e;
+        bool valid = key < p.Nk;
+        if (valid && p.mask != nullptr) valid = p.mask[b * p.mask_sb + (int64_t)key * p.mask_sk] != 0;
+        if (!valid) inv |= 1u << e;
+      }
+      const uint32_t any = __ballot_sync(0xffffffffu, inv != 0);
+      const int t = j % kBiasStages;
+      for (int w = 0; w < kQTiles && ok; ++w) {
+        const int slot = w * kBiasStages + t;
+        ok = mbar_wait(&bars[L::kBarBiasFull + slot], (j / kBiasStages) & 1, wc);
+        if (!ok) break;
+        if (any) {
+          uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
+          uint32_t rem = any;
+          while (rem) {
+            const int src = __ffs(rem) - 1;
+            rem &= rem - 1;
+            const uint32_t bits = __shfl_sync(0xffffffffu, inv, src);
+            for (int e = 0; e < 4; ++e) {
+              if (!((bits >> e) & 1u)) continue;
+              const int c = 4 * src + e;  // key column inside the tile
+              if (kBiasT) {
+                // row c of the [key][query] tile: 128 bf16 = 256 bytes
+                uint2 *row = reinterpret_cast<uint2 *>(tile + c * 256);
+                row[lane] = make_uint2(0xFF80FF80u, 0xFF80FF80u);
+              } else {
+                const int box = c >> 6, cc = c & 63, chunk = cc >> 3, el = cc & 7;
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) {
+                  const int r = lane + 32 * rr;
+                  uint16_t *ptr = reinterpret_cast<uint16_t *>(tile + box * (L::kBiasBytes / 2) + r * 128 +
+                                                               ((chunk ^ (r & 7)) << 4) + el * 2);
+                  *ptr = 0xFF80u;  // bf16 -inf
+                }
+              }
+            }
+          }
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        mbar_arrive(&bars[L::kBarBiasReady + slot]);
+      }
+    }
+  } else {
+    // ================================================================ softmax warpgroups
+    const int w = warp >> 2;            // query tile
+    const int t = threadIdx.x & 127;    // row inside the tile
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + w * kBN;
+    const uint32_t tP = tmem + lane_base + 256 + w * 64;
+    const uint32_t tO = tmem + lane_base + 384 + w * 64;
+    const float tau = p.tau;
+    float m_cur = -INFINITY;   // maximum used for P and l
+    float m_true = -INFINITY;  // true running maximum
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt && ok; ++j) {
+      ok = mbar_wait(&bars[L::kBarSFull + w], j & 1, wc);
+      if (!ok) break;
+      tc_fence_after_sync();
+      uint32_t sreg[kBN];
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sreg[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before_sync();
+      mbar_arrive(&bars[L::kBarSFree + w]);
+
+      const int slot = w * kBiasStages + (j % kBiasStages);
+      ok = mbar_wait(&bars[(p.needs_mask ? L::kBarBiasReady : L::kBarBiasFull) + slot], (j / kBiasStages) & 1, wc);
+      if (!ok) break;
+      const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
+      float x[kBN];
+      if (kBiasT) {
+        const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
+#pragma unroll
+        for (int c = 0; c < kBN; ++c)
+          x[c] = fmaf(__uint_as_float(sreg[c]), tau, __uint_as_float(uint32_t(col[c * kBM]) << 16));
+      } else {
+#pragma unroll
+        for (int c8 = 0; c8 < kBN / 8; ++c8) {
+          const int box = c8 >> 3, chunk = c8 & 7;
+          const uint4 bv = *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 +
+                                                            ((chunk ^ (t & 7)) << 4));
+          const uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x[c8 * 8 + 2 * e] = fmaf(__uint_as_float(sreg[c8 * 8 + 2 * e]), tau, bf16lo_to_f32(wv[e]));
+            x[c8 * 8 + 2 * e + 1] = fmaf(__uint_as_float(sreg[c8 * 8 + 2 * e + 1]), tau, bf16hi_to_f32(wv[e]));
+          }
+        }
+      }
+      mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
+
+      // tile maximum
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBN; c += 2) mx = max3f(mx, x[c], x[c + 1]);
+      m_true = fmaxf(m_true, mx);
+      const bool need = mx > m_cur + kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = (m_cur == -INFINITY) ? 0.f : ex2_approx((m_cur - mx) * kLog2e);
+        l *= alpha;
+        m_cur = mx;
+      }
+      const float neg_m = (m_cur == -INFINITY) ? 0.f : -m_cur * kLog2e;
+      uint32_t pk[kBN / 2];
+      float lsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBN; c += 2) {
+        const float p0 = ex2_approx(fmaf(x[c], kLog2e, neg_m));
+        const float p1 = ex2_approx(fmaf(x[c + 1], kLog2e, neg_m));
+        lsum += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l += lsum;
+
+      if (j > 0) {
+        ok = mbar_wait(&bars[L::kBarODone + w], (j - 1) & 1, wc);
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (__any_sync(0xffffffffu, need)) {
+          // rescale this warp's rows of O (lanes without a new maximum use 1)
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c, o);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kBN / 2; c += 32) tmem_st32(tP + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&bars[L::kBarPFull + w]);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    if (ok) ok = mbar_wait(&bars[L::kBarODone + w], (nt - 1) & 1, wc);
+    if (ok) {
+      tc_fence_after_sync();
+      const int row = q0 + w * kBM + t;
+      float o[D];
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tO + c, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[c + e] = __uint_as_float(r[e]);
+      }
+      if (row < p.Nq) {
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        if (kEpi == kEpiForward) {
+          float g[D];
+          if (kGate) {
+            const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + b * p.gate_sb + h * p.gate_sh +
+                                                              (int64_t)row * p.gate_sn);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c) {
+              const uint4 gv = gp[c];
+              const uint32_t wv[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                g[c * 8 + 2 * e] = bf16lo_to_f32(wv[e]);
+                g[c * 8 + 2 * e + 1] = bf16hi_to_f32(wv[e]);
+              }
+            }
+          }
+          uint4 *op = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + b * p.out_sb + h * p.out_sh +
+                                                (int64_t)row * p.out_sn);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float v0 = o[c * 8 + 2 * e] * inv_l, v1 = o[c * 8 + 2 * e + 1] * inv_l;
+              if (kGate) {
+                v0 *= 1.f / (1.f + __expf(-g[c * 8 + 2 * e]));
+                v1 *= 1.f / (1.f + __expf(-g[c * 8 + 2 * e + 1]));
+              }
+              wv[e] = pack_bf16x2(v0, v1);
+            }
+            op[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+          if (p.lse != nullptr)
+            p.lse[b * p.lse_sb + h * p.lse_sh + (int64_t)row * p.lse_sn] = (l > 0.f) ? m_cur + logf(l) : -INFINITY;
+        } else {
+          float4 *op = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + b * p.out_sb + h * p.out_sh +
+                                                  (int64_t)row * p.out_sn);
+#pragma unroll
+          for (int c = 0; c < D / 4; ++c)
+            op[c] = make_float4(o[4 * c] * inv_l, o[4 * c + 1] * inv_l, o[4 * c + 2] * inv_l, o[4 * c + 3] * inv_l);
+          const int64_t mi = b * p.lse_sb + h * p.lse_sh + (int64_t)row * p.lse_sn;
+          p.lse[mi] = (l > 0.f) ? m_true : -INFINITY;
+          p.l_part[mi] = (l > 0.f) ? l * ex2_approx((m_cur - m_true) * kLog2e) : 0.f;
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace pba
