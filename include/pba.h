@@ -31,6 +31,8 @@
  *     l = 0 for partials); never NaN.  Values of K and V must be finite,
  *     masked keys included.  NaN or +inf in the inputs is outside the
  *     contract.
+ *   - A pointer may be NULL when the tensor it stands for has no element
+ *     (Nq = 0 or Nk = 0); every other required pointer must be non-NULL.
  *   - Return values: PBA_OK when the launch was enqueued.  PBA_ERR_INVALID_ARG
  *     for a NULL required pointer, a negative size, a misaligned pointer or
  *     stride (see below), or a size beyond the limits.  PBA_ERR_UNSUPPORTED for

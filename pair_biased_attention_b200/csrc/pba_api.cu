@@ -116,6 +116,13 @@ cudaError_t launch_tc(const pba::AttnParams &p, int grid, cudaStream_t stream) {
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+    // The kernel moves registers between its warpgroups with setmaxnreg; the
+    // split must fit in what the block is launched with, or the increase
+    // would wait forever.  Refuse to launch a build where it would not.
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+        fa.numRegs * pba::kAttnThreads < pba::kRegSplitTotal)
+      attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kAttnThreads, L::kSmemAlloc, stream>>>(p);
@@ -236,8 +243,12 @@ pba_status attn_common(const pba_attn_desc *d, const void *q, const void *k, con
                        const uint8_t *mask, bool partial, void *out, float *lse, float *l_part, void *stream_ptr) {
   pba_status s = check_desc(d);
   if (s != PBA_OK) return s;
-  if (q == nullptr || k == nullptr || v == nullptr || bias == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
-  if (partial && (lse == nullptr || l_part == nullptr)) return PBA_ERR_INVALID_ARG;
+  // a pointer may be NULL only when the tensor it stands for has no element
+  const bool has_q = d->Nq > 0, has_k = d->Nk > 0;
+  if ((has_q && (q == nullptr || out == nullptr)) || (has_k && (k == nullptr || v == nullptr)) ||
+      (has_q && has_k && bias == nullptr))
+    return PBA_ERR_INVALID_ARG;
+  if (has_q && partial && (lse == nullptr || l_part == nullptr)) return PBA_ERR_INVALID_ARG;
   s = check_device();
   if (s != PBA_OK) return s;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);

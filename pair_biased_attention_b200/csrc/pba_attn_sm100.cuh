@@ -15,8 +15,8 @@
 // One CTA per SM holds two 128-row query tiles of one (b, h):
 //   warps 0-3   softmax warpgroup for query tile 0 (thread t owns row t)
 //   warps 4-7   softmax warpgroup for query tile 1
-//   warp 8      TMA producer: Q once, then K, V and the two bias tiles per
-//               128-key tile, through shared-memory rings
+//   warp 8      TMA producer of Q (once) and of K, V per 128-key tile
+//   warp 11     TMA producer of the two bias tiles per 128-key tile
 //   warp 9      allocates Tensor Memory and issues every tcgen05.mma
 //   warp 10     key-mask warp: writes -inf into the bias tile columns of
 //               masked keys and of keys past the end, in shared memory, before
@@ -39,11 +39,16 @@ constexpr int kBM = 128;          // query rows per tile (one TMEM lane each)
 constexpr int kBN = 128;          // keys per tile
 constexpr int kQTiles = 2;        // query tiles per CTA
 constexpr int kBiasStages = 2;    // bias ring depth per softmax warpgroup
-constexpr int kAttnThreads = 352; // 11 warps
-constexpr int kWarpProducer = 8;
+constexpr int kAttnThreads = 384; // 12 warps
+constexpr int kWarpProducer = 8;  // Q, K, V
 constexpr int kWarpMma = 9;
 constexpr int kWarpMask = 10;
+constexpr int kWarpBiasProducer = 11;
 constexpr uint32_t kTmemCols = 512;
+// Per-thread register limits after the warpgroup reallocation.
+constexpr int kRegsSoftmax = 216;
+constexpr int kRegsOther = 56;
+constexpr int kRegSplitTotal = 256 * kRegsSoftmax + 128 * kRegsOther;
 
 enum Epilogue : int { kEpiForward = 0, kEpiPartial = 1 };
 
@@ -163,12 +168,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
-    tma_prefetch_desc(&p.tm_bias);
   }
+  if (warp == kWarpBiasProducer && lane == 0) tma_prefetch_desc(&p.tm_bias);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+
   const WaitCtl wc{abort_flag, p.err, p.timeout_ns};
   WaitCtl wc_drain = wc;  // clean-up waits: ignore the abort word, keep the time limit
   int drain_abort = 0;
@@ -177,6 +183,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
   const int hb = p.bias_h_bcast ? 0 : h;
   const int bb = p.bias_b_bcast ? 0 : b;
 
+  // Registers: the launch gives 168 per thread (384 x 168 = 64512).  The
+  // producer/MMA/mask warpgroup (warps 8-11) gives most of its share to the
+  // two softmax warpgroups: 128 x 56 + 256 x 216 = 62464 <= 64512.  Each
+  // warpgroup changes its limit once, at the top of its own branch.
+  if (warp >= 8) {
+  setmaxnreg_dec<kRegsOther>();
   if (warp == kWarpProducer) {
     // ================================================================ TMA producer
     if (lane == 0) {
@@ -184,7 +196,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       const uint64_t pol_keep = l2_policy_evict_last();
       bool ok = true;
       // times each full barrier was armed, for the clean-up on abort
-      int arms_k[L::kKVStages] = {}, arms_v[L::kKVStages] = {}, arms_b[kQTiles * kBiasStages] = {};
+      int arms_k[L::kKVStages] = {}, arms_v[L::kKVStages] = {};
       mbar_arrive_expect_tx(&bars[L::kBarQFull], kQTiles * L::kQBytes);
       for (int w = 0; w < kQTiles; ++w)
         tma_load_4d(smem + L::kOffQ + w * L::kQBytes, &p.tm_q, &bars[L::kBarQFull], 0, q0 + w * kBM, h, b,
@@ -201,6 +213,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         tma_load_4d(smem + L::kOffV + s * L::kKVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kBN, h, b,
                     pol_keep);
         ++arms_v[s];
+      }
+      if (!ok) {
+        // Let every copy already issued land before the CTA exits: each full
+        // barrier has at most one armed phase that no consumer has waited for.
+        mbar_wait(&bars[L::kBarQFull], 0, wc_drain);
+        for (int s = 0; s < L::kKVStages; ++s) {
+          if (arms_k[s]) mbar_wait(&bars[L::kBarKFull + s], (arms_k[s] - 1) & 1, wc_drain);
+          if (arms_v[s]) mbar_wait(&bars[L::kBarVFull + s], (arms_v[s] - 1) & 1, wc_drain);
+        }
+      }
+    }
+  } else if (warp == kWarpBiasProducer) {
+    // ================================================================ bias TMA producer
+    if (lane == 0) {
+      const uint64_t pol_stream = l2_policy_evict_first();
+      bool ok = true;
+      int arms_b[kQTiles * kBiasStages] = {};
+      for (int j = 0; j < nt && ok; ++j) {
         const int t = j % kBiasStages;
         for (int w = 0; w < kQTiles && ok; ++w) {
           const int slot = w * kBiasStages + t;
@@ -220,17 +250,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           ++arms_b[slot];
         }
       }
-      if (!ok) {
-        // Let every copy already issued land before the CTA exits: each full
-        // barrier has at most one armed phase that no consumer has waited for.
-        mbar_wait(&bars[L::kBarQFull], 0, wc_drain);
-        for (int s = 0; s < L::kKVStages; ++s) {
-          if (arms_k[s]) mbar_wait(&bars[L::kBarKFull + s], (arms_k[s] - 1) & 1, wc_drain);
-          if (arms_v[s]) mbar_wait(&bars[L::kBarVFull + s], (arms_v[s] - 1) & 1, wc_drain);
-        }
+      if (!ok)
         for (int i = 0; i < kQTiles * kBiasStages; ++i)
           if (arms_b[i]) mbar_wait(&bars[L::kBarBiasFull + i], (arms_b[i] - 1) & 1, wc_drain);
-      }
     }
   } else if (warp == kWarpMma) {
     // ================================================================ MMA issuer
@@ -348,8 +370,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         mbar_arrive(&bars[L::kBarBiasReady + slot]);
       }
     }
+  }
   } else {
     // ================================================================ softmax warpgroups
+    setmaxnreg_inc<kRegsSoftmax>();
     const int w = warp >> 2;            // query tile
     const int t = threadIdx.x & 127;    // row inside the tile
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
@@ -376,12 +400,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       ok = mbar_wait(&bars[(p.needs_mask ? L::kBarBiasReady : L::kBarBiasFull) + slot], (j / kBiasStages) & 1, wc);
       if (!ok) break;
       const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
-      float x[kBN];
+      // x = tau * s + bias, two keys per packed fma
+      float2 x[kBN / 2];
+      const float2 tau2 = make_float2(tau, tau);
       if (kBiasT) {
         const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
 #pragma unroll
-        for (int c = 0; c < kBN; ++c)
-          x[c] = fmaf(__uint_as_float(sreg[c]), tau, __uint_as_float(uint32_t(col[c * kBM]) << 16));
+        for (int c = 0; c < kBN; c += 2) {
+          const float2 bv = make_float2(__uint_as_float(uint32_t(col[c * kBM]) << 16),
+                                        __uint_as_float(uint32_t(col[(c + 1) * kBM]) << 16));
+          x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2, bv);
+        }
       } else {
 #pragma unroll
         for (int c8 = 0; c8 < kBN / 8; ++c8) {
@@ -391,17 +420,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           const uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            x[c8 * 8 + 2 * e] = fmaf(__uint_as_float(sreg[c8 * 8 + 2 * e]), tau, bf16lo_to_f32(wv[e]));
-            x[c8 * 8 + 2 * e + 1] = fmaf(__uint_as_float(sreg[c8 * 8 + 2 * e + 1]), tau, bf16hi_to_f32(wv[e]));
+            const int c = c8 * 8 + 2 * e;
+            x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2,
+                             make_float2(bf16lo_to_f32(wv[e]), bf16hi_to_f32(wv[e])));
           }
         }
       }
       mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
 
-      // tile maximum
-      float mx = -INFINITY;
+      // tile maximum: four independent chains
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) mx = max3f(mx, x[c], x[c + 1]);
+      for (int i = 0; i < kBN / 2; ++i) m4[i & 3] = max3f(m4[i & 3], x[i].x, x[i].y);
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       m_true = fmaxf(m_true, mx);
       const bool need = mx > m_cur + kRescaleThreshold;
       float alpha = 1.f;
@@ -411,16 +442,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         m_cur = mx;
       }
       const float neg_m = (m_cur == -INFINITY) ? 0.f : -m_cur * kLog2e;
+      const float2 l2e2 = make_float2(kLog2e, kLog2e), negm2 = make_float2(neg_m, neg_m);
       uint32_t pk[kBN / 2];
-      float lsum = 0.f;
+      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < kBN; c += 2) {
-        const float p0 = ex2_approx(fmaf(x[c], kLog2e, neg_m));
-        const float p1 = ex2_approx(fmaf(x[c + 1], kLog2e, neg_m));
-        lsum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+      for (int i = 0; i < kBN / 2; ++i) {
+        const float2 a = ffma2(x[i], l2e2, negm2);
+        const float2 pv = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+        ls[i & 3] = fadd2(ls[i & 3], pv);
+        pk[i] = pack_bf16x2(pv.x, pv.y);
       }
-      l += lsum;
+      const float2 lsum2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+      l += lsum2.x + lsum2.y;
 
       if (j > 0) {
         ok = mbar_wait(&bars[L::kBarODone + w], (j - 1) & 1, wc);
