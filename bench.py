@@ -57,6 +57,31 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def kernel_source_sha256() -> str:
+    import glob
+    import hashlib
+
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "pair_biased_attention_b200", "csrc", "*.cu*")))
+    for f in files + [os.path.join(ROOT, "include", "pba.h")]:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """DRAM bytes per large16k launch from the last ncu capture, or None when
+    the kernel sources changed since that capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    if rec.get("kernel_source_sha256") != kernel_source_sha256():
+        return None
+    return rec.get("pba_attn_sm100_large16k_bytes_per_launch")
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -74,7 +99,7 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
 
@@ -153,34 +178,30 @@ def barrier(pg: bool):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_sample(q, k, v, bias, mask, target_s=10.0, max_rows=4096):
-    """Times the fp64 oracle on a bounded sample of query rows of the large
-    workload (all 16384 keys each).  Returns (TFLOP/s, threads, description)."""
+def oracle_sample(q, k, v, bias, mask, target_s=10.0, chunk_rows=1024):
+    """Times the fp64 oracle on sampled query rows of the large workload (all
+    16384 keys each), one chunk of rows per head round robin, until about
+    target_s seconds of oracle time.  Returns (TFLOP/s, threads, description,
+    seconds)."""
     import oracle
 
     H, N, D = q.shape[1], q.shape[2], q.shape[3]
     g = torch.Generator("cpu").manual_seed(77)
-
-    def run(nrows):
-        per_head = max(1, nrows // H)
-        flops, t = 0.0, 0.0
-        for h in range(H):
-            rows = torch.randperm(N, generator=g)[:per_head].to(q.device)
-            qs = q[:, h:h + 1].index_select(2, rows).cpu()
-            bs = bias[:, h:h + 1].index_select(2, rows).cpu()
-            ks, vs = k[:, h:h + 1].cpu(), v[:, h:h + 1].cpu()
-            ms = None if mask is None else mask.cpu()
-            t0 = time.perf_counter()
-            oracle.pba(qs, ks, vs, bs, ms)
-            t += time.perf_counter() - t0
-            flops += attn_flops(1, 1, per_head, N, D)
-        return flops, t, per_head * H
-
-    f, t, n = run(H * 4)
-    rate = f / t
-    want = int(min(max_rows, max(H, target_s * rate / attn_flops(1, 1, 1, N, D))))
-    f, t, n = run(want)
-    return f / t / 1e12, oracle.threads_used(), f"{n} query rows x {N} keys of large16k (fp64 oracle, sampled rows)", t
+    flops, t, nrows, h = 0.0, 0.0, 0, 0
+    ms = None if mask is None else mask.cpu()
+    while t < target_s and nrows < 64 * chunk_rows:
+        rows = torch.randperm(N, generator=g)[:chunk_rows].to(q.device)
+        qs = q[:, h:h + 1].index_select(2, rows).cpu()
+        bs = bias[:, h:h + 1].index_select(2, rows).cpu()
+        ks, vs = k[:, h:h + 1].cpu(), v[:, h:h + 1].cpu()
+        t0 = time.perf_counter()
+        oracle.pba(qs, ks, vs, bs, ms)
+        t += time.perf_counter() - t0
+        flops += attn_flops(1, 1, chunk_rows, N, D)
+        nrows += chunk_rows
+        h = (h + 1) % H
+    return (flops / t / 1e12, oracle.threads_used(),
+            f"{nrows} query rows x {N} keys of large16k, {chunk_rows}-row chunks over the heads (fp64 oracle)", t)
 
 
 # ------------------------------------------------------------------ the reference arm
@@ -235,7 +256,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -309,11 +330,7 @@ def main():
     tri_rows_per_s = world * tri_rows * args.steps / (t_tri / 1e3)
     tri_flops = 2 * attn_flops(tcfg.N, tcfg.H, tcfg.N, tcfg.N, tcfg.D)
 
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            traffic = json.load(f).get("pba_attn_sm100_large16k_bytes_per_launch")
+    traffic = measured_traffic()
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -199,6 +199,16 @@ PBA_API uint64_t pba_set_wait_timeout_ns(uint64_t timeout_ns);
  */
 PBA_API pba_status pba_selftest_wait_timeout(uint64_t timeout_ns, void *stream);
 
+/*
+ * pba_selftest_exp2 -- applies the kernels' software 2^x (the share of the
+ * exponentials computed on the FMA pipe instead of the exp2 unit) to n floats:
+ * out[i] = 2^in[i], in and out device arrays.  Range reduction 2^n * 2^f with
+ * a degree-4 polynomial for 2^f on [-1/2, 1/2]; relative error below 1e-5 for
+ * inputs in [-126, 128); inputs at or below -127 (and -inf) give exactly 0.
+ * No counterpart on the pages: it lets tests check that approximation.
+ */
+PBA_API pba_status pba_selftest_exp2(const float *in, float *out, int64_t n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

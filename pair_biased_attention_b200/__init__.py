@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "PbaError", "PBA_OK", "PBA_ERR_INVALID_ARG", "PBA_ERR_UNSUPPORTED", "PBA_ERR_CUDA", "PBA_ERR_TIMEOUT",
     "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward",
-    "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_status_string",
+    "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_selftest_exp2",
+    "pba_status_string",
 ]
 
 PBA_OK, PBA_ERR_INVALID_ARG, PBA_ERR_UNSUPPORTED, PBA_ERR_CUDA, PBA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -88,6 +89,8 @@ def load_library() -> ctypes.CDLL:
     lib.pba_set_wait_timeout_ns.restype = ctypes.c_uint64
     lib.pba_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _p]
     lib.pba_selftest_wait_timeout.restype = st
+    lib.pba_selftest_exp2.argtypes = [_p, _p, ctypes.c_int64, _p]
+    lib.pba_selftest_exp2.restype = st
     _LIB = lib
     return lib
 
@@ -282,6 +285,17 @@ def pba_last_device_error(stream=None) -> int:
 
 def pba_set_wait_timeout_ns(ns: int) -> int:
     return load_library().pba_set_wait_timeout_ns(int(ns))
+
+
+def pba_selftest_exp2(x, out=None, stream=None):
+    """The kernels' software 2^x applied to a CUDA fp32 tensor (test hook)."""
+    _cuda("x", x, torch.float32)
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if out is None:
+        out = torch.empty_like(x)
+    _check("pba_selftest_exp2", load_library().pba_selftest_exp2(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
+    return out
 
 
 def pba_selftest_wait_timeout(ns: int, stream=None) -> None:

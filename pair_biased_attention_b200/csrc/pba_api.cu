@@ -108,10 +108,10 @@ struct TcProblem {
   int64_t gate_s[3];
 };
 
-template <int D, bool kBiasT, int kEpi, bool kGate>
+template <int D, bool kBiasT, int kEpi, bool kGate, bool kMasked>
 cudaError_t launch_tc(const pba::AttnParams &p, int grid, cudaStream_t stream) {
   using L = pba::AttnLayout<D>;
-  auto kern = pba::pba_attn_sm100_kernel<D, kBiasT, kEpi, kGate>;
+  auto kern = pba::pba_attn_sm100_kernel<D, kBiasT, kEpi, kGate, kMasked>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -129,13 +129,23 @@ cudaError_t launch_tc(const pba::AttnParams &p, int grid, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Instantiations: untransposed bias tiles with and without key masking
+// (masked keys and a ragged key tail are applied as mask words), transposed
+// bias tiles (triangle attention, ending node; masking by the mask warp).
 template <int D>
 cudaError_t dispatch_tc(const pba::AttnParams &p, int grid, bool bias_t, int epi, bool gate, cudaStream_t st) {
-  if (epi == pba::kEpiPartial) return launch_tc<D, false, pba::kEpiPartial, false>(p, grid, st);
-  if (!bias_t && !gate) return launch_tc<D, false, pba::kEpiForward, false>(p, grid, st);
-  if (!bias_t && gate) return launch_tc<D, false, pba::kEpiForward, true>(p, grid, st);
-  if (bias_t && !gate) return launch_tc<D, true, pba::kEpiForward, false>(p, grid, st);
-  return launch_tc<D, true, pba::kEpiForward, true>(p, grid, st);
+  const bool m = p.needs_mask != 0;
+  if (epi == pba::kEpiPartial)
+    return m ? launch_tc<D, false, pba::kEpiPartial, false, true>(p, grid, st)
+             : launch_tc<D, false, pba::kEpiPartial, false, false>(p, grid, st);
+  if (bias_t)
+    return gate ? launch_tc<D, true, pba::kEpiForward, true, false>(p, grid, st)
+                : launch_tc<D, true, pba::kEpiForward, false, false>(p, grid, st);
+  if (gate)
+    return m ? launch_tc<D, false, pba::kEpiForward, true, true>(p, grid, st)
+             : launch_tc<D, false, pba::kEpiForward, true, false>(p, grid, st);
+  return m ? launch_tc<D, false, pba::kEpiForward, false, true>(p, grid, st)
+           : launch_tc<D, false, pba::kEpiForward, false, false>(p, grid, st);
 }
 
 pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
@@ -177,6 +187,8 @@ pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
   p.bias_h_bcast = t.bias_h_bcast;
   p.bias_b_bcast = t.bias_b_bcast;
   p.needs_mask = (t.mask != nullptr) || (t.Nk % pba::kBN != 0);
+  p.mask_vec4 = t.mask != nullptr && t.mask_sk == 1 && (reinterpret_cast<uintptr_t>(t.mask) & 3u) == 0 &&
+                t.mask_sb % 4 == 0;
   p.tau = t.tau;
   p.mask = t.mask;
   p.mask_sb = t.mask_sb;
@@ -482,6 +494,15 @@ pba_status pba_selftest_wait_timeout(uint64_t timeout_ns, void *stream) {
   int *err = device_error_word();
   if (err == nullptr) return PBA_ERR_CUDA;
   pba::pba_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+pba_status pba_selftest_exp2(const float *in, float *out, int64_t n, void *stream) {
+  if (n < 0 || (n > 0 && (in == nullptr || out == nullptr))) return PBA_ERR_INVALID_ARG;
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  if (n == 0) return PBA_OK;
+  pba::pba_exp2_selftest_kernel<<<148, 256, 0, static_cast<cudaStream_t>(stream)>>>(in, out, n);
   return cudaGetLastError() == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
 }
 

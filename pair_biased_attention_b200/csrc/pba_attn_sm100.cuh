@@ -59,6 +59,7 @@ struct AttnParams {
   int32_t bias_h_bcast;  // bias head stride 0
   int32_t bias_b_bcast;  // bias batch stride 0
   int32_t needs_mask;    // key mask given or Nk not a multiple of the key tile
+  int32_t mask_vec4;     // key mask rows readable as aligned 4-byte words
   float tau;
   const uint8_t *mask;
   int64_t mask_sb, mask_sk;
@@ -87,13 +88,16 @@ struct AttnLayout {
   static constexpr int kOffK = kOffQ + kQTiles * kQBytes;
   static constexpr int kOffV = kOffK + kKVStages * kKVBytes;
   static constexpr int kOffBias = kOffV + kKVStages * kKVBytes;
-  static constexpr int kOffBar = kOffBias + kQTiles * kBiasStages * kBiasBytes;
+  // key-mask words: one u32 per key pair of a bias slot (0xFFFF per valid half)
+  static constexpr int kOffMaskWords = kOffBias + kQTiles * kBiasStages * kBiasBytes;
+  static constexpr int kOffBar = kOffMaskWords + kQTiles * kBiasStages * (kBN / 2) * 4;
   // barriers
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKFull = 1;
   static constexpr int kBarVFull = kBarKFull + kKVStages;
-  static constexpr int kBarKVEmpty = kBarVFull + kKVStages;
-  static constexpr int kBarBiasFull = kBarKVEmpty + kKVStages;            // [w][t]
+  static constexpr int kBarKEmpty = kBarVFull + kKVStages;
+  static constexpr int kBarVEmpty = kBarKEmpty + kKVStages;
+  static constexpr int kBarBiasFull = kBarVEmpty + kKVStages;             // [w][t]
   static constexpr int kBarBiasReady = kBarBiasFull + kQTiles * kBiasStages;
   static constexpr int kBarBiasEmpty = kBarBiasReady + kQTiles * kBiasStages;
   static constexpr int kBarSFull = kBarBiasEmpty + kQTiles * kBiasStages;  // [w]
@@ -116,10 +120,20 @@ constexpr float kLog2e = 1.4426950408889634f;
 // maximum is used consistently for P and l, so the result is unchanged and the
 // probabilities stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f / kLog2e;
+// One key pair in kExpEmuEvery takes the software exp2 (0: none).  At D = 32
+// the exp2 unit is the tighter limit and a third of the pairs move to the FMA
+// pipe; at D = 64 the softmax is issue-bound and all pairs use the unit.
+#ifndef PBA_EXP_EMU_EVERY_D32
+#define PBA_EXP_EMU_EVERY_D32 3
+#endif
+#ifndef PBA_EXP_EMU_EVERY_D64
+#define PBA_EXP_EMU_EVERY_D64 0
+#endif
 
-template <int D, bool kBiasT, int kEpi, bool kGate>
+template <int D, bool kBiasT, int kEpi, bool kGate, bool kMasked>
 __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const __grid_constant__ AttnParams p) {
   using L = AttnLayout<D>;
+  constexpr int kExpEmuEvery = (D == 32) ? PBA_EXP_EMU_EVERY_D32 : PBA_EXP_EMU_EVERY_D64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
@@ -143,7 +157,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
     for (int s = 0; s < L::kKVStages; ++s) {
       mbar_init(&bars[L::kBarKFull + s], 1);
       mbar_init(&bars[L::kBarVFull + s], 1);
-      mbar_init(&bars[L::kBarKVEmpty + s], 1);
+      mbar_init(&bars[L::kBarKEmpty + s], 1);
+      mbar_init(&bars[L::kBarVEmpty + s], 1);
     }
     for (int i = 0; i < kQTiles * kBiasStages; ++i) {
       mbar_init(&bars[L::kBarBiasFull + i], 1);
@@ -201,18 +216,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       for (int w = 0; w < kQTiles; ++w)
         tma_load_4d(smem + L::kOffQ + w * L::kQBytes, &p.tm_q, &bars[L::kBarQFull], 0, q0 + w * kBM, h, b,
                     pol_stream);
-      for (int j = 0; j < nt && ok; ++j) {
+      // K runs one tile ahead of V: a K slot frees when both score MMAs of its
+      // tile are done, a V slot only after both P V MMAs.
+      auto load_k = [&](int j) -> bool {
         const int s = j % L::kKVStages;
-        if (j >= L::kKVStages) ok = mbar_wait(&bars[L::kBarKVEmpty + s], ((j / L::kKVStages) - 1) & 1, wc);
-        if (!ok) break;
+        if (j >= L::kKVStages && !mbar_wait(&bars[L::kBarKEmpty + s], ((j / L::kKVStages) - 1) & 1, wc))
+          return false;
         mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kKVBytes);
         tma_load_4d(smem + L::kOffK + s * L::kKVBytes, &p.tm_k, &bars[L::kBarKFull + s], 0, j * kBN, h, b,
                     pol_keep);
         ++arms_k[s];
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int s = j % L::kKVStages;
+        if (j >= L::kKVStages && !mbar_wait(&bars[L::kBarVEmpty + s], ((j / L::kKVStages) - 1) & 1, wc))
+          return false;
         mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kKVBytes);
         tma_load_4d(smem + L::kOffV + s * L::kKVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kBN, h, b,
                     pol_keep);
         ++arms_v[s];
+        return true;
+      };
+      ok = load_k(0);
+      for (int j = 0; j < nt && ok; ++j) {
+        if (j + 1 < nt) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
       }
       if (!ok) {
         // Let every copy already issued land before the CTA exits: each full
@@ -286,32 +315,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         }
         tc_commit(&bars[L::kBarODone + w]);
       };
-      for (int j = 0; j < nt && ok; ++j) {
+      // Issue order: S0(j+1), S1(j+1) as soon as each softmax warpgroup has
+      // read S(j), then P0 V(j), P1 V(j).  The next score tiles are computed
+      // while the softmax warpgroups work on tile j.
+      auto issue_s_pair = [&](int j) -> bool {
         const int s = j % L::kKVStages;
-        ok = mbar_wait(&bars[L::kBarKFull + s], (j / L::kKVStages) & 1, wc);
-        for (int w = 0; w < kQTiles && ok; ++w) {
-          if (j > 0) ok = mbar_wait(&bars[L::kBarSFree + w], (j - 1) & 1, wc);
-          if (!ok) break;
+        if (!mbar_wait(&bars[L::kBarKFull + s], (j / L::kKVStages) & 1, wc)) return false;
+        for (int w = 0; w < kQTiles; ++w) {
+          if (j > 0 && !mbar_wait(&bars[L::kBarSFree + w], (j - 1) & 1, wc)) return false;
           tc_fence_after_sync();
           issue_s(w, j);
-          if (j > 0) {
-            const int sp = (j - 1) % L::kKVStages;
-            ok = mbar_wait(&bars[L::kBarPFull + w], (j - 1) & 1, wc) &&
-                 mbar_wait(&bars[L::kBarVFull + sp], ((j - 1) / L::kKVStages) & 1, wc);
-            if (!ok) break;
-            tc_fence_after_sync();
-            issue_pv(w, j - 1);
-            if (w == kQTiles - 1) tc_commit(&bars[L::kBarKVEmpty + sp]);
-          }
         }
-      }
-      for (int w = 0; w < kQTiles && ok; ++w) {
-        const int sp = (nt - 1) % L::kKVStages;
-        ok = mbar_wait(&bars[L::kBarPFull + w], (nt - 1) & 1, wc) &&
-             mbar_wait(&bars[L::kBarVFull + sp], ((nt - 1) / L::kKVStages) & 1, wc);
+        tc_commit(&bars[L::kBarKEmpty + s]);
+        return true;
+      };
+      if (ok) ok = issue_s_pair(0);
+      for (int j = 0; j < nt && ok; ++j) {
+        if (j + 1 < nt) ok = issue_s_pair(j + 1);
         if (!ok) break;
-        tc_fence_after_sync();
-        issue_pv(w, nt - 1);
+        const int s = j % L::kKVStages;
+        ok = mbar_wait(&bars[L::kBarVFull + s], (j / L::kKVStages) & 1, wc);
+        for (int w = 0; w < kQTiles && ok; ++w) {
+          ok = mbar_wait(&bars[L::kBarPFull + w], j & 1, wc);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_pv(w, j);
+        }
+        if (ok) tc_commit(&bars[L::kBarVEmpty + s]);
       }
       // Every MMA issued above completes before Tensor Memory is released.
       tc_commit(&bars[L::kBarDrain]);
@@ -319,49 +349,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
     }
   } else if (warp == kWarpMask) {
     // ================================================================ key-mask warp
+    // Lane l owns keys 4l..4l+3 of each tile; the mask bytes of tile j+1 are
+    // loaded while tile j is processed.  For the untransposed bias tile the
+    // warp writes one mask word per key pair beside the bias slot and the
+    // softmax warps apply it while unpacking the bias; for the transposed
+    // tile (one key per 256-byte row) it writes -inf over the masked rows.
     // Without a key mask and with whole key tiles the softmax warps wait on
     // the TMA barrier directly and this warp has nothing to do.
-    bool ok = p.needs_mask != 0;
-    for (int j = 0; j < nt && ok; ++j) {
-      const int k0 = j * kBN;
-      uint32_t inv = 0;  // bit e: key k0 + 4*lane + e is masked or past the end
+    bool ok = kBiasT ? (p.needs_mask != 0) : kMasked;
+    const uint8_t *mrow = p.mask ? p.mask + (int64_t)b * p.mask_sb : nullptr;
+    auto load_word = [&](int j) -> uint32_t {  // byte e nonzero = key 4*lane+e takes part
+      const int key0 = j * kBN + 4 * lane;
+      if (mrow == nullptr) return 0x01010101u;
+      if (p.mask_vec4 && key0 + 3 < p.Nk) return __ldg(reinterpret_cast<const uint32_t *>(mrow + key0));
+      uint32_t wv = 0;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = k0 + 4 * lane + e;
-        bool valid = key < p.Nk;
-        if (valid && p.mask != nullptr) valid = p.mask[b * p.mask_sb + (int64_t)key * p.mask_sk] != 0;
-        if (!valid) inv |= 1u << e;
-      }
-      const uint32_t any = __ballot_sync(0xffffffffu, inv != 0);
+      for (int e = 0; e < 4; ++e)
+        if (key0 + e < p.Nk) wv |= uint32_t(__ldg(mrow + (int64_t)(key0 + e) * p.mask_sk) != 0) << (8 * e);
+      return wv;
+    };
+    uint32_t next_word = ok ? load_word(0) : 0u;
+    for (int j = 0; j < nt && ok; ++j) {
+      const uint32_t word = next_word;
+      if (j + 1 < nt) next_word = load_word(j + 1);
+      const int key0 = j * kBN + 4 * lane;
+      uint32_t inv = 0;  // bit e: key 4*lane + e of the tile is masked or past the end
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (key0 + e >= p.Nk || ((word >> (8 * e)) & 0xFFu) == 0) inv |= 1u << e;
+      // keep-masks of the key pairs (4l, 4l+1) and (4l+2, 4l+3)
+      const uint2 keep = make_uint2(((inv & 1u) ? 0u : 0x0000FFFFu) | ((inv & 2u) ? 0u : 0xFFFF0000u),
+                                    ((inv & 4u) ? 0u : 0x0000FFFFu) | ((inv & 8u) ? 0u : 0xFFFF0000u));
+      const uint32_t any = kBiasT ? __ballot_sync(0xffffffffu, inv != 0) : 0u;
       const int t = j % kBiasStages;
       for (int w = 0; w < kQTiles && ok; ++w) {
         const int slot = w * kBiasStages + t;
         ok = mbar_wait(&bars[L::kBarBiasFull + slot], (j / kBiasStages) & 1, wc);
         if (!ok) break;
-        if (any) {
+        if (!kBiasT) {
+          reinterpret_cast<uint2 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[lane] = keep;
+        } else if (any) {
           uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
           uint32_t rem = any;
           while (rem) {
             const int src = __ffs(rem) - 1;
             rem &= rem - 1;
-            const uint32_t bits = __shfl_sync(0xffffffffu, inv, src);
-            for (int e = 0; e < 4; ++e) {
-              if (!((bits >> e) & 1u)) continue;
-              const int c = 4 * src + e;  // key column inside the tile
-              if (kBiasT) {
-                // row c of the [key][query] tile: 128 bf16 = 256 bytes
-                uint2 *row = reinterpret_cast<uint2 *>(tile + c * 256);
-                row[lane] = make_uint2(0xFF80FF80u, 0xFF80FF80u);
-              } else {
-                const int box = c >> 6, cc = c & 63, chunk = cc >> 3, el = cc & 7;
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr) {
-                  const int r = lane + 32 * rr;
-                  uint16_t *ptr = reinterpret_cast<uint16_t *>(tile + box * (L::kBiasBytes / 2) + r * 128 +
-                                                               ((chunk ^ (r & 7)) << 4) + el * 2);
-                  *ptr = 0xFF80u;  // bf16 -inf
-                }
-              }
+            uint32_t bits = __shfl_sync(0xffffffffu, inv, src);
+            while (bits) {
+              const int e = __ffs(bits) - 1;
+              bits &= bits - 1;
+              // row 4*src+e of the [key][query] tile: 128 bf16 = 256 bytes
+              reinterpret_cast<uint2 *>(tile + (4 * src + e) * 256)[lane] = make_uint2(0xFF80FF80u, 0xFF80FF80u);
             }
           }
           fence_proxy_async_smem();
@@ -397,7 +435,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       mbar_arrive(&bars[L::kBarSFree + w]);
 
       const int slot = w * kBiasStages + (j % kBiasStages);
-      ok = mbar_wait(&bars[(p.needs_mask ? L::kBarBiasReady : L::kBarBiasFull) + slot], (j / kBiasStages) & 1, wc);
+      const bool relay = kBiasT ? (p.needs_mask != 0) : kMasked;
+      ok = mbar_wait(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (j / kBiasStages) & 1, wc);
       if (!ok) break;
       const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
       // x = tau * s + bias, two keys per packed fma
@@ -417,7 +456,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           const int box = c8 >> 3, chunk = c8 & 7;
           const uint4 bv = *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 +
                                                             ((chunk ^ (t & 7)) << 4));
-          const uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
+          uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
+          if (kMasked) {
+            // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
+            const uint4 kv = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
+            const uint32_t keep[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) wv[e] = (wv[e] & keep[e]) | (~keep[e] & 0xFF80FF80u);
+          }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c8 * 8 + 2 * e;
@@ -428,11 +474,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       }
       mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
 
-      // tile maximum: four independent chains
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // tile maximum: eight independent chains
+      float m8[8];
 #pragma unroll
-      for (int i = 0; i < kBN / 2; ++i) m4[i & 3] = max3f(m4[i & 3], x[i].x, x[i].y);
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(x[i].x, x[i].y);
+#pragma unroll
+      for (int i = 8; i < kBN / 2; ++i) m8[i & 7] = max3f(m8[i & 7], x[i].x, x[i].y);
+      const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       m_true = fmaxf(m_true, mx);
       const bool need = mx > m_cur + kRescaleThreshold;
       float alpha = 1.f;
@@ -448,7 +496,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
 #pragma unroll
       for (int i = 0; i < kBN / 2; ++i) {
         const float2 a = ffma2(x[i], l2e2, negm2);
-        const float2 pv = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+        // every kExpEmuEvery-th key pair takes the software exp2 on the FMA pipe
+        const float2 pv = (kExpEmuEvery > 0 && i % kExpEmuEvery == kExpEmuEvery - 1)
+                              ? exp2_poly2(a)
+                              : make_float2(ex2_approx(a.x), ex2_approx(a.y));
         ls[i & 3] = fadd2(ls[i & 3], pv);
         pk[i] = pack_bf16x2(pv.x, pv.y);
       }

@@ -54,6 +54,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Longest time (ns) a waiting thread may stay suspended in one try_wait.
+#ifndef PBA_WAIT_HINT_NS
+#define PBA_WAIT_HINT_NS 20000u
+#endif
+
+// As mbar_try_wait, but the thread may stay suspended up to `hint_ns`
+// nanoseconds; it resumes as soon as the phase completes.  Cuts the issue
+// slots a waiting warp spends polling.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Per-CTA wait control: a shared abort word and the time limit.  A wait that
 // runs out sets the abort word and records kErrTimeout in the device error
 // word; every other wait in the CTA sees the abort word and gives up too, so
@@ -69,8 +88,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
   const uint64_t t0 = global_timer_ns();
   uint32_t iter = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++iter & 15u) == 0) {
+    if (PBA_WAIT_HINT_NS ? mbar_try_wait_hint(bar, parity, PBA_WAIT_HINT_NS) : mbar_try_wait(bar, parity))
+      return true;
+    if ((++iter & 3u) == 0) {
       if (*w.abort_flag) return false;
       if (global_timer_ns() - t0 > w.timeout_ns) {
         *w.abort_flag = 1;
@@ -237,6 +257,15 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 // Packed fp32 pairs (one instruction for two lanes of math).
+#ifndef PBA_PACKED_F32X2
+#define PBA_PACKED_F32X2 1
+#endif
+#if !PBA_PACKED_F32X2
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return make_float2(a.x + b.x, a.y + b.y); }
+#else
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   float2 d;
   asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -253,6 +282,44 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+#endif
+
+// Software 2^x for a pair, on the FMA pipe (the exp2 unit is the scarce one).
+// Cody-Waite reduction 2^x = 2^n * 2^f, n = round(x), f = x - n in [-1/2, 1/2];
+// 2^f by the degree-4 polynomial 1 + c1 f + ... + c4 f^4 whose coefficients
+// minimise the relative error on [-1/2, 1/2] with the constant term held at 1
+// (fitted by fit_exp2_poly.py; max relative error 2.9e-6 in fp32; integer
+// arguments give exact powers of two).  n comes from adding 1.5*2^23 + 127: the low mantissa bits of the sum
+// hold n + 127, which shifted into the exponent field is the fp32 value 2^n.
+// Inputs are clamped at -127, where that scale is exactly 0, so -inf (a
+// masked key) and everything below 2^-127 give 0, as the hardware exp2 with
+// flush-to-zero does.  Inputs above 128 are outside its range (the softmax
+// never passes more than 8).
+__device__ __forceinline__ float2 exp2_poly2(float2 a) {
+  a.x = fmaxf(a.x, -127.f);
+  a.y = fmaxf(a.y, -127.f);
+  const float2 shift = make_float2(12583039.f, 12583039.f);  // 1.5 * 2^23 + 127
+  const float2 t = fadd2(a, shift);
+  const float2 n = fadd2(t, make_float2(-12583039.f, -12583039.f));
+  const float2 f = fadd2(a, make_float2(-n.x, -n.y));
+  float2 q = ffma2(make_float2(9.582576342e-03f, 9.582576342e-03f), f,
+                   make_float2(5.590682849e-02f, 5.590682849e-02f));
+  q = ffma2(q, f, make_float2(2.402410656e-01f, 2.402410656e-01f));
+  q = ffma2(q, f, make_float2(6.931241155e-01f, 6.931241155e-01f));
+  q = ffma2(q, f, make_float2(1.0f, 1.0f));
+  const float2 scale = make_float2(__uint_as_float(__float_as_uint(t.x) << 23),
+                                   __uint_as_float(__float_as_uint(t.y) << 23));
+  return fmul2(q, scale);
 }
 
 // Two fp32 values -> packed bf16x2 (round to nearest even); `lo` in bits [0,16).

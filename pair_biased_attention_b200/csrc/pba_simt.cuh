@@ -193,6 +193,16 @@ __global__ void pba_empty_keys_kernel(const EmptyParams p) {
   }
 }
 
+// Applies the attention kernel's software exp2 (exp2_poly2) to n values.
+__global__ void pba_exp2_selftest_kernel(const float *in, float *out, int64_t n) {
+  for (int64_t i = 2 * (int64_t(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+       i += 2 * int64_t(gridDim.x) * blockDim.x) {
+    const float2 r = exp2_poly2(make_float2(in[i], i + 1 < n ? in[i + 1] : 0.f));
+    out[i] = r.x;
+    if (i + 1 < n) out[i + 1] = r.y;
+  }
+}
+
 // Waits on a barrier that no thread ever completes; the bounded wait must give
 // up after timeout_ns and record kErrTimeout.
 __global__ void pba_wait_selftest_kernel(int *err, uint64_t timeout_ns) {

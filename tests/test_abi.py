@@ -29,7 +29,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "pba_status_string",
-              "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout"):
+              "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout",
+              "pba_selftest_exp2"):
         assert n in names
 
 
