@@ -158,14 +158,21 @@ def dist_setup(args):
     return world, rank, local, pg
 
 
-def max_over_ranks(x: float, pg: bool) -> float:
+def max_over_ranks(x: float, pg: bool, device: str = "cuda") -> float:
+    """Largest value over the ranks (the step time every rank waits for)."""
     if not pg:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, work_per_rank_step: float, steps: int, t_max_ms: float) -> float:
+    """Whole-job rate: every rank does the same work per step (weak scaling);
+    the job time is the slowest rank's."""
+    return world * work_per_rank_step * steps / (t_max_ms / 1e3)
 
 
 def barrier(pg: bool):
@@ -323,11 +330,11 @@ def main():
 
     flops = attn_flops(cfg.B, cfg.H, cfg.N, cfg.N, cfg.D)
     nbytes = attn_bytes(cfg.B, cfg.H, cfg.N, cfg.N, cfg.D)
-    value = world * flops * args.steps / (t_pba / 1e3) / 1e12
+    value = job_throughput(world, flops, args.steps, t_pba) / 1e12
     avg_launch_s = sum(pba_ms) / len(pba_ms) / 1e3
     achieved_gbs = nbytes / avg_launch_s / 1e9
     tri_rows = 2 * tcfg.N  # pair-tensor rows per step (starting + ending)
-    tri_rows_per_s = world * tri_rows * args.steps / (t_tri / 1e3)
+    tri_rows_per_s = job_throughput(world, tri_rows, args.steps, t_tri)
     tri_flops = 2 * attn_flops(tcfg.N, tcfg.H, tcfg.N, tcfg.N, tcfg.D)
 
     traffic = measured_traffic()
