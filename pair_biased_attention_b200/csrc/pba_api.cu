@@ -184,6 +184,9 @@ pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
   p.Nq = t.Nq;
   p.Nk = t.Nk;
   p.n_qblocks = (t.Nq + pba::kQTiles * pba::kBM - 1) / (pba::kQTiles * pba::kBM);
+  const int64_t n_units = int64_t(t.B) * t.H * p.n_qblocks;
+  if (n_units > kMaxI32) return PBA_ERR_INVALID_ARG;
+  p.n_units = int(n_units);
   p.bias_h_bcast = t.bias_h_bcast;
   p.bias_b_bcast = t.bias_b_bcast;
   p.needs_mask = (t.mask != nullptr) || (t.Nk % pba::kBN != 0);
@@ -209,8 +212,15 @@ pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
   p.err = device_error_word();
   if (p.err == nullptr) return PBA_ERR_CUDA;
   p.timeout_ns = g_timeout_ns.load();
-  const int64_t grid = int64_t(t.B) * t.H * p.n_qblocks;
-  if (grid > kMaxI32) return PBA_ERR_INVALID_ARG;
+  // persistent: one CTA per SM (each needs most of the SM's shared memory)
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return PBA_ERR_CUDA;
+#ifndef PBA_PERSISTENT_GRID
+#define PBA_PERSISTENT_GRID 1
+#endif
+  const int64_t grid = (PBA_PERSISTENT_GRID && n_units > sms) ? sms : n_units;
   cudaError_t e = (t.D == 64) ? dispatch_tc<64>(p, int(grid), t.bias_t, t.epi, t.gate != nullptr, stream)
                               : dispatch_tc<32>(p, int(grid), t.bias_t, t.epi, t.gate != nullptr, stream);
   return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;

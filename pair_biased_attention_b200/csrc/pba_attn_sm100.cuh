@@ -2,8 +2,8 @@
 //
 // Computes, per (batch b, head h) and query row i,
 //     O_i = sum_j softmax_j( tau q_i.k_j + b_ij ) v_j
-// over the key tiles of one call, as in "Fold-CP: A Context Parallelism
-// Framework for Biomolecular Modeling" (Table 1 "Attn Pair Bias", Figure 2(c):
+// over the keys of one call, as in "Fold-CP: A Context Parallelism Framework
+// for Biomolecular Modeling" (Table 1 "Attn Pair Bias", Figure 2(c):
 // attention of the local queries against a key/value/pair-bias block).  The
 // softmax is accumulated online, tile by tile (the method of "Online
 // normalizer calculation for softmax", listed under "Builds on" on the
@@ -12,21 +12,24 @@
 // O_p, m_p, l_p that the tiled-softmax merge combines).  Triangle attention
 // runs the same loop with the pair-tensor strides in the tile descriptors.
 //
-// One CTA per SM holds two 128-row query tiles of one (b, h):
+// Persistent: one CTA per SM walks the work units u = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; a unit is two 128-row query tiles of one
+// (b, h).  Every ring and barrier phase runs on across units, so the next
+// unit's Q, K, V and bias loads overlap the current unit's last tiles and
+// epilogue.
 //   warps 0-3   softmax warpgroup for query tile 0 (thread t owns row t)
 //   warps 4-7   softmax warpgroup for query tile 1
-//   warp 8      TMA producer of Q (once) and of K, V per 128-key tile
-//   warp 11     TMA producer of the two bias tiles per 128-key tile
+//   warp 8      TMA producer of Q (per unit) and of K, V per 128-key tile
 //   warp 9      allocates Tensor Memory and issues every tcgen05.mma
-//   warp 10     key-mask warp: writes -inf into the bias tile columns of
-//               masked keys and of keys past the end, in shared memory, before
-//               the softmax warps read the tile
+//   warp 10     key-mask warp (mask words, or -inf rows of a transposed tile)
+//   warp 11     TMA producer of the two bias tiles per 128-key tile
 // Tensor Memory (512 columns x 128 lanes of fp32):
 //   [0,128) S0   [128,256) S1   [256,320) P0   [320,384) P1
 //   [384,384+D) O0   [448,448+D) O1
 // S_w = Q_w K^T (fp32), P_w = bf16 probabilities (two per column), O_w the
-// running output.  The MMA warp issues S0(j), PV0(j-1), S1(j), PV1(j-1), so
-// the next score tile is computed while the softmax warps work on this one.
+// running output.  MMA issue order per key tile j: S0(j+1), P0 V(j), S1(j+1),
+// P1 V(j), so the next score tile is computed while the softmax warps work
+// on this one.
 #pragma once
 
 #include <cuda.h>
@@ -37,7 +40,7 @@ namespace pba {
 
 constexpr int kBM = 128;          // query rows per tile (one TMEM lane each)
 constexpr int kBN = 128;          // keys per tile
-constexpr int kQTiles = 2;        // query tiles per CTA
+constexpr int kQTiles = 2;        // query tiles per unit
 constexpr int kBiasStages = 2;    // bias ring depth per softmax warpgroup
 constexpr int kAttnThreads = 384; // 12 warps
 constexpr int kWarpProducer = 8;  // Q, K, V
@@ -46,7 +49,7 @@ constexpr int kWarpMask = 10;
 constexpr int kWarpBiasProducer = 11;
 constexpr uint32_t kTmemCols = 512;
 // Per-thread register limits after the warpgroup reallocation.
-constexpr int kRegsSoftmax = 216;
+constexpr int kRegsSoftmax = 224;
 constexpr int kRegsOther = 56;
 constexpr int kRegSplitTotal = 256 * kRegsSoftmax + 128 * kRegsOther;
 
@@ -56,6 +59,7 @@ struct AttnParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_bias;
   int32_t B, H, Nq, Nk;
   int32_t n_qblocks;     // ceil(Nq / 256)
+  int32_t n_units;       // B * H * n_qblocks
   int32_t bias_h_bcast;  // bias head stride 0
   int32_t bias_b_bcast;  // bias batch stride 0
   int32_t needs_mask;    // key mask given or Nk not a multiple of the key tile
@@ -93,7 +97,8 @@ struct AttnLayout {
   static constexpr int kOffBar = kOffMaskWords + kQTiles * kBiasStages * (kBN / 2) * 4;
   // barriers
   static constexpr int kBarQFull = 0;
-  static constexpr int kBarKFull = 1;
+  static constexpr int kBarQEmpty = 1;
+  static constexpr int kBarKFull = 2;
   static constexpr int kBarVFull = kBarKFull + kKVStages;
   static constexpr int kBarKEmpty = kBarVFull + kKVStages;
   static constexpr int kBarVEmpty = kBarKEmpty + kKVStages;
@@ -104,7 +109,8 @@ struct AttnLayout {
   static constexpr int kBarSFree = kBarSFull + kQTiles;
   static constexpr int kBarPFull = kBarSFree + kQTiles;
   static constexpr int kBarODone = kBarPFull + kQTiles;
-  static constexpr int kBarDrain = kBarODone + kQTiles;
+  static constexpr int kBarOFree = kBarODone + kQTiles;  // [w]: epilogue has read O
+  static constexpr int kBarDrain = kBarOFree + kQTiles;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemSlot + 4;
@@ -130,6 +136,17 @@ constexpr float kRescaleThreshold = 8.0f / kLog2e;
 #define PBA_EXP_EMU_EVERY_D64 0
 #endif
 
+// Work unit u -> (b, h, first query row); units are ordered query block
+// fastest, then head, then batch, so concurrent CTAs share one head's K/V.
+struct Unit {
+  int b, h, q0;
+};
+__device__ __forceinline__ Unit decode_unit(const AttnParams &p, int u) {
+  const int qblk = u % p.n_qblocks;
+  const int bh = u / p.n_qblocks;
+  return Unit{bh / p.H, bh % p.H, qblk * (kQTiles * kBM)};
+}
+
 template <int D, bool kBiasT, int kEpi, bool kGate, bool kMasked>
 __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const __grid_constant__ AttnParams p) {
   using L = AttnLayout<D>;
@@ -142,18 +159,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work unit: (b, h, 256 query rows)
-  const int unit = blockIdx.x;
-  const int qblk = unit % p.n_qblocks;
-  const int bh = unit / p.n_qblocks;
-  const int h = bh % p.H;
-  const int b = bh / p.H;
-  const int q0 = qblk * (kQTiles * kBM);
-  const int nt = (p.Nk + kBN - 1) / kBN;
+  const int nt = (p.Nk + kBN - 1) / kBN;  // key tiles per unit
+  const int u_begin = blockIdx.x, u_step = gridDim.x;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[L::kBarQFull], 1);
+    mbar_init(&bars[L::kBarQEmpty], 1);
     for (int s = 0; s < L::kKVStages; ++s) {
       mbar_init(&bars[L::kBarKFull + s], 1);
       mbar_init(&bars[L::kBarVFull + s], 1);
@@ -170,6 +181,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       mbar_init(&bars[L::kBarSFree + w], kBM);
       mbar_init(&bars[L::kBarPFull + w], kBM);
       mbar_init(&bars[L::kBarODone + w], 1);
+      mbar_init(&bars[L::kBarOFree + w], kBM);
     }
     mbar_init(&bars[L::kBarDrain], 1);
     *abort_flag = 0;
@@ -189,226 +201,275 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-
   const WaitCtl wc{abort_flag, p.err, p.timeout_ns};
   WaitCtl wc_drain = wc;  // clean-up waits: ignore the abort word, keep the time limit
   int drain_abort = 0;
   wc_drain.abort_flag = &drain_abort;
 
-  const int hb = p.bias_h_bcast ? 0 : h;
-  const int bb = p.bias_b_bcast ? 0 : b;
-
   // Registers: the launch gives 168 per thread (384 x 168 = 64512).  The
   // producer/MMA/mask warpgroup (warps 8-11) gives most of its share to the
-  // two softmax warpgroups: 128 x 56 + 256 x 216 = 62464 <= 64512.  Each
+  // two softmax warpgroups: 128 x 56 + 256 x 224 = 64512.  Each
   // warpgroup changes its limit once, at the top of its own branch.
   if (warp >= 8) {
-  setmaxnreg_dec<kRegsOther>();
-  if (warp == kWarpProducer) {
-    // ================================================================ TMA producer
-    if (lane == 0) {
-      const uint64_t pol_stream = l2_policy_evict_first();
-      const uint64_t pol_keep = l2_policy_evict_last();
-      bool ok = true;
-      // times each full barrier was armed, for the clean-up on abort
-      int arms_k[L::kKVStages] = {}, arms_v[L::kKVStages] = {};
-      mbar_arrive_expect_tx(&bars[L::kBarQFull], kQTiles * L::kQBytes);
-      for (int w = 0; w < kQTiles; ++w)
-        tma_load_4d(smem + L::kOffQ + w * L::kQBytes, &p.tm_q, &bars[L::kBarQFull], 0, q0 + w * kBM, h, b,
-                    pol_stream);
-      // K runs one tile ahead of V: a K slot frees when both score MMAs of its
-      // tile are done, a V slot only after both P V MMAs.
-      auto load_k = [&](int j) -> bool {
-        const int s = j % L::kKVStages;
-        if (j >= L::kKVStages && !mbar_wait(&bars[L::kBarKEmpty + s], ((j / L::kKVStages) - 1) & 1, wc))
-          return false;
-        mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kKVBytes);
-        tma_load_4d(smem + L::kOffK + s * L::kKVBytes, &p.tm_k, &bars[L::kBarKFull + s], 0, j * kBN, h, b,
-                    pol_keep);
-        ++arms_k[s];
-        return true;
-      };
-      auto load_v = [&](int j) -> bool {
-        const int s = j % L::kKVStages;
-        if (j >= L::kKVStages && !mbar_wait(&bars[L::kBarVEmpty + s], ((j / L::kKVStages) - 1) & 1, wc))
-          return false;
-        mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kKVBytes);
-        tma_load_4d(smem + L::kOffV + s * L::kKVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kBN, h, b,
-                    pol_keep);
-        ++arms_v[s];
-        return true;
-      };
-      ok = load_k(0);
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt) ok = load_k(j + 1);
-        if (ok) ok = load_v(j);
-      }
-      if (!ok) {
-        // Let every copy already issued land before the CTA exits: each full
-        // barrier has at most one armed phase that no consumer has waited for.
-        mbar_wait(&bars[L::kBarQFull], 0, wc_drain);
-        for (int s = 0; s < L::kKVStages; ++s) {
-          if (arms_k[s]) mbar_wait(&bars[L::kBarKFull + s], (arms_k[s] - 1) & 1, wc_drain);
-          if (arms_v[s]) mbar_wait(&bars[L::kBarVFull + s], (arms_v[s] - 1) & 1, wc_drain);
-        }
-      }
-    }
-  } else if (warp == kWarpBiasProducer) {
-    // ================================================================ bias TMA producer
-    if (lane == 0) {
-      const uint64_t pol_stream = l2_policy_evict_first();
-      bool ok = true;
-      int arms_b[kQTiles * kBiasStages] = {};
-      for (int j = 0; j < nt && ok; ++j) {
-        const int t = j % kBiasStages;
-        for (int w = 0; w < kQTiles && ok; ++w) {
-          const int slot = w * kBiasStages + t;
-          if (j >= kBiasStages) ok = mbar_wait(&bars[L::kBarBiasEmpty + slot], ((j / kBiasStages) - 1) & 1, wc);
+    setmaxnreg_dec<kRegsOther>();
+    if (warp == kWarpProducer) {
+      // ============================================================== Q/K/V TMA producer
+      if (lane == 0) {
+        const uint64_t pol_stream = l2_policy_evict_first();
+        const uint64_t pol_keep = l2_policy_evict_last();
+        bool ok = true;
+        int kc = 0, vc = 0, uc = 0, qc = 0;  // K tiles, V tiles, units, Q loads issued
+        // K runs one tile ahead of V: a K slot frees when both score MMAs of its
+        // tile are done, a V slot only after both P V MMAs.
+        auto load_k = [&](const Unit &un, int j) -> bool {
+          const int s = kc % L::kKVStages;
+          if (kc >= L::kKVStages && !mbar_wait(&bars[L::kBarKEmpty + s], ((kc / L::kKVStages) - 1) & 1, wc))
+            return false;
+          mbar_arrive_expect_tx(&bars[L::kBarKFull + s], L::kKVBytes);
+          tma_load_4d(smem + L::kOffK + s * L::kKVBytes, &p.tm_k, &bars[L::kBarKFull + s], 0, j * kBN, un.h, un.b,
+                      pol_keep);
+          ++kc;
+          return true;
+        };
+        auto load_v = [&](const Unit &un, int j) -> bool {
+          const int s = vc % L::kKVStages;
+          if (vc >= L::kKVStages && !mbar_wait(&bars[L::kBarVEmpty + s], ((vc / L::kKVStages) - 1) & 1, wc))
+            return false;
+          mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kKVBytes);
+          tma_load_4d(smem + L::kOffV + s * L::kKVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kBN, un.h, un.b,
+                      pol_keep);
+          ++vc;
+          return true;
+        };
+        for (int u = u_begin; u < p.n_units && ok; u += u_step, ++uc) {
+          const Unit un = decode_unit(p, u);
+          // Q slot: free once the last score MMAs of the previous unit are done
+          if (uc > 0) ok = mbar_wait(&bars[L::kBarQEmpty], (uc - 1) & 1, wc);
           if (!ok) break;
-          uint8_t *dst = smem + L::kOffBias + slot * L::kBiasBytes;
-          mbar_arrive_expect_tx(&bars[L::kBarBiasFull + slot], L::kBiasBytes);
-          if (kBiasT) {
-            // transposed bias tile: [128 keys][128 queries], no swizzle
-            tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], q0 + w * kBM, j * kBN, hb, bb, pol_stream);
-          } else {
-            // [128 queries][128 keys] as two 64-key boxes, 128-byte swizzle
-            tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN, q0 + w * kBM, hb, bb, pol_stream);
-            tma_load_4d(dst + L::kBiasBytes / 2, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN + 64,
-                        q0 + w * kBM, hb, bb, pol_stream);
+          mbar_arrive_expect_tx(&bars[L::kBarQFull], kQTiles * L::kQBytes);
+          for (int w = 0; w < kQTiles; ++w)
+            tma_load_4d(smem + L::kOffQ + w * L::kQBytes, &p.tm_q, &bars[L::kBarQFull], 0, un.q0 + w * kBM, un.h,
+                        un.b, pol_stream);
+          ++qc;
+          ok = load_k(un, 0);
+          for (int j = 0; j < nt && ok; ++j) {
+            if (j + 1 < nt) ok = load_k(un, j + 1);
+            if (ok) ok = load_v(un, j);
           }
-          ++arms_b[slot];
+        }
+        if (!ok) {
+          // Let every copy already issued land before the CTA exits: each full
+          // barrier has at most one armed phase that no consumer has waited for.
+          // slot s was armed (n - s + stages - 1) / stages times after n issues
+          if (qc) mbar_wait(&bars[L::kBarQFull], (qc - 1) & 1, wc_drain);
+          for (int s = 0; s < L::kKVStages; ++s) {
+            const int ak = (kc - s + L::kKVStages - 1) / L::kKVStages, av = (vc - s + L::kKVStages - 1) / L::kKVStages;
+            if (ak > 0) mbar_wait(&bars[L::kBarKFull + s], (ak - 1) & 1, wc_drain);
+            if (av > 0) mbar_wait(&bars[L::kBarVFull + s], (av - 1) & 1, wc_drain);
+          }
         }
       }
-      if (!ok)
-        for (int i = 0; i < kQTiles * kBiasStages; ++i)
-          if (arms_b[i]) mbar_wait(&bars[L::kBarBiasFull + i], (arms_b[i] - 1) & 1, wc_drain);
-    }
-  } else if (warp == kWarpMma) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);
-      const uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
-      const uint32_t sQ = smem_u32(smem + L::kOffQ);
-      const uint32_t sK = smem_u32(smem + L::kOffK);
-      const uint32_t sV = smem_u32(smem + L::kOffV);
-      bool ok = mbar_wait(&bars[L::kBarQFull], 0, wc);
-      auto issue_s = [&](int w, int j) {
-        const int s = j % L::kKVStages;
-        const uint32_t d_tmem = tmem + w * kBN;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = smem_desc(sQ + w * L::kQBytes + kk * 32, 16, L::kAtomBytes, L::kSwizzleMode);
-          const uint64_t bdesc = smem_desc(sK + s * L::kKVBytes + kk * 32, 16, L::kAtomBytes, L::kSwizzleMode);
-          mma_bf16_ss(d_tmem, a, bdesc, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars[L::kBarSFull + w]);
-      };
-      auto issue_pv = [&](int w, int j) {
-        const int s = j % L::kKVStages;
-        const uint32_t d_tmem = tmem + 384 + w * 64;
-        const uint32_t a_tmem = tmem + 256 + w * 64;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bdesc = smem_desc(sV + s * L::kKVBytes + kk * 16 * L::kRowBytes, L::kKVBytes, L::kAtomBytes,
-                                           L::kSwizzleMode);
-          mma_bf16_ts(d_tmem, a_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bars[L::kBarODone + w]);
-      };
-      // Issue order: S0(j+1), S1(j+1) as soon as each softmax warpgroup has
-      // read S(j), then P0 V(j), P1 V(j).  The next score tiles are computed
-      // while the softmax warpgroups work on tile j.
-      auto issue_s_pair = [&](int j) -> bool {
-        const int s = j % L::kKVStages;
-        if (!mbar_wait(&bars[L::kBarKFull + s], (j / L::kKVStages) & 1, wc)) return false;
-        for (int w = 0; w < kQTiles; ++w) {
-          if (j > 0 && !mbar_wait(&bars[L::kBarSFree + w], (j - 1) & 1, wc)) return false;
-          tc_fence_after_sync();
-          issue_s(w, j);
-        }
-        tc_commit(&bars[L::kBarKEmpty + s]);
-        return true;
-      };
-      if (ok) ok = issue_s_pair(0);
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt) ok = issue_s_pair(j + 1);
-        if (!ok) break;
-        const int s = j % L::kKVStages;
-        ok = mbar_wait(&bars[L::kBarVFull + s], (j / L::kKVStages) & 1, wc);
-        for (int w = 0; w < kQTiles && ok; ++w) {
-          ok = mbar_wait(&bars[L::kBarPFull + w], j & 1, wc);
-          if (!ok) break;
-          tc_fence_after_sync();
-          issue_pv(w, j);
-        }
-        if (ok) tc_commit(&bars[L::kBarVEmpty + s]);
-      }
-      // Every MMA issued above completes before Tensor Memory is released.
-      tc_commit(&bars[L::kBarDrain]);
-      mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
-    }
-  } else if (warp == kWarpMask) {
-    // ================================================================ key-mask warp
-    // Lane l owns keys 4l..4l+3 of each tile; the mask bytes of tile j+1 are
-    // loaded while tile j is processed.  For the untransposed bias tile the
-    // warp writes one mask word per key pair beside the bias slot and the
-    // softmax warps apply it while unpacking the bias; for the transposed
-    // tile (one key per 256-byte row) it writes -inf over the masked rows.
-    // Without a key mask and with whole key tiles the softmax warps wait on
-    // the TMA barrier directly and this warp has nothing to do.
-    bool ok = kBiasT ? (p.needs_mask != 0) : kMasked;
-    const uint8_t *mrow = p.mask ? p.mask + (int64_t)b * p.mask_sb : nullptr;
-    auto load_word = [&](int j) -> uint32_t {  // byte e nonzero = key 4*lane+e takes part
-      const int key0 = j * kBN + 4 * lane;
-      if (mrow == nullptr) return 0x01010101u;
-      if (p.mask_vec4 && key0 + 3 < p.Nk) return __ldg(reinterpret_cast<const uint32_t *>(mrow + key0));
-      uint32_t wv = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (key0 + e < p.Nk) wv |= uint32_t(__ldg(mrow + (int64_t)(key0 + e) * p.mask_sk) != 0) << (8 * e);
-      return wv;
-    };
-    uint32_t next_word = ok ? load_word(0) : 0u;
-    for (int j = 0; j < nt && ok; ++j) {
-      const uint32_t word = next_word;
-      if (j + 1 < nt) next_word = load_word(j + 1);
-      const int key0 = j * kBN + 4 * lane;
-      uint32_t inv = 0;  // bit e: key 4*lane + e of the tile is masked or past the end
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (key0 + e >= p.Nk || ((word >> (8 * e)) & 0xFFu) == 0) inv |= 1u << e;
-      // keep-masks of the key pairs (4l, 4l+1) and (4l+2, 4l+3)
-      const uint2 keep = make_uint2(((inv & 1u) ? 0u : 0x0000FFFFu) | ((inv & 2u) ? 0u : 0xFFFF0000u),
-                                    ((inv & 4u) ? 0u : 0x0000FFFFu) | ((inv & 8u) ? 0u : 0xFFFF0000u));
-      const uint32_t any = kBiasT ? __ballot_sync(0xffffffffu, inv != 0) : 0u;
-      const int t = j % kBiasStages;
-      for (int w = 0; w < kQTiles && ok; ++w) {
-        const int slot = w * kBiasStages + t;
-        ok = mbar_wait(&bars[L::kBarBiasFull + slot], (j / kBiasStages) & 1, wc);
-        if (!ok) break;
-        if (!kBiasT) {
-          reinterpret_cast<uint2 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[lane] = keep;
-        } else if (any) {
-          uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
-          uint32_t rem = any;
-          while (rem) {
-            const int src = __ffs(rem) - 1;
-            rem &= rem - 1;
-            uint32_t bits = __shfl_sync(0xffffffffu, inv, src);
-            while (bits) {
-              const int e = __ffs(bits) - 1;
-              bits &= bits - 1;
-              // row 4*src+e of the [key][query] tile: 128 bf16 = 256 bytes
-              reinterpret_cast<uint2 *>(tile + (4 * src + e) * 256)[lane] = make_uint2(0xFF80FF80u, 0xFF80FF80u);
+    } else if (warp == kWarpBiasProducer) {
+      // ============================================================== bias TMA producer
+      if (lane == 0) {
+        const uint64_t pol_stream = l2_policy_evict_first();
+        bool ok = true;
+        int gt = 0;      // key tiles started (all units)
+        int issued = 0;  // bias tiles issued, warpgroup-major within a key tile
+        for (int u = u_begin; u < p.n_units && ok; u += u_step) {
+          const Unit un = decode_unit(p, u);
+          const int hb = p.bias_h_bcast ? 0 : un.h;
+          const int bb = p.bias_b_bcast ? 0 : un.b;
+          for (int j = 0; j < nt && ok; ++j, ++gt) {
+            const int t = gt % kBiasStages;
+            for (int w = 0; w < kQTiles && ok; ++w) {
+              const int slot = w * kBiasStages + t;
+              if (gt >= kBiasStages)
+                ok = mbar_wait(&bars[L::kBarBiasEmpty + slot], ((gt / kBiasStages) - 1) & 1, wc);
+              if (!ok) break;
+              uint8_t *dst = smem + L::kOffBias + slot * L::kBiasBytes;
+              mbar_arrive_expect_tx(&bars[L::kBarBiasFull + slot], L::kBiasBytes);
+              if (kBiasT) {
+                // transposed bias tile: [128 keys][128 queries], no swizzle
+                tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], un.q0 + w * kBM, j * kBN, hb, bb,
+                            pol_stream);
+              } else {
+                // [128 queries][128 keys] as two 64-key boxes, 128-byte swizzle
+                tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN, un.q0 + w * kBM, hb, bb,
+                            pol_stream);
+                tma_load_4d(dst + L::kBiasBytes / 2, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN + 64,
+                            un.q0 + w * kBM, hb, bb, pol_stream);
+              }
+              ++issued;
             }
           }
-          fence_proxy_async_smem();
         }
-        __syncwarp();
-        mbar_arrive(&bars[L::kBarBiasReady + slot]);
+        if (!ok)
+          for (int w = 0; w < kQTiles; ++w)
+            for (int t = 0; t < kBiasStages; ++t) {
+              // tiles of warpgroup w issued: key tiles 0..n_w-1, slot t armed for those with tile % stages == t
+              const int n_w = issued / kQTiles + (w < issued % kQTiles ? 1 : 0);
+              const int a = (n_w - t + kBiasStages - 1) / kBiasStages;
+              if (a > 0) mbar_wait(&bars[L::kBarBiasFull + w * kBiasStages + t], (a - 1) & 1, wc_drain);
+            }
+      }
+    } else if (warp == kWarpMma) {
+      // ============================================================== MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc_s = idesc_bf16_f32(kBM, kBN, false);
+        const uint32_t idesc_o = idesc_bf16_f32(kBM, D, true);
+        const uint32_t sQ = smem_u32(smem + L::kOffQ);
+        const uint32_t sK = smem_u32(smem + L::kOffK);
+        const uint32_t sV = smem_u32(smem + L::kOffV);
+        bool ok = true;
+        int kc = 0, vc = 0;  // K and V tiles consumed
+        int gs = 0;          // score tiles issued (all units), per warpgroup
+        int gp = 0;          // P V tiles issued (all units), per warpgroup
+        int uc = 0;
+        // Descriptor high halves are fixed; the loops advance the address field
+        // of the low half (16 bytes per unit): 32 bytes per K step inside a
+        // swizzle row of Q and K, 16 key rows per K step down V.
+        constexpr uint32_t kDescHi = smem_desc_hi(L::kAtomBytes, L::kSwizzleMode);
+        auto issue_s = [&](int w, int s) {
+          const uint32_t d_tmem = tmem + w * kBN;
+          const uint32_t a_lo = smem_desc_lo(sQ + w * L::kQBytes, 16);
+          const uint32_t b_lo = smem_desc_lo(sK + s * L::kKVBytes, 16);
+#pragma unroll 4
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(d_tmem, desc_join(a_lo + kk * 2, kDescHi), desc_join(b_lo + kk * 2, kDescHi), idesc_s,
+                        kk > 0 ? 1u : 0u);
+          tc_commit(&bars[L::kBarSFull + w]);
+        };
+        auto issue_pv = [&](int w, int s, bool first) {
+          const uint32_t d_tmem = tmem + 384 + w * 64;
+          const uint32_t a_tmem = tmem + 256 + w * 64;
+          const uint32_t v_lo = smem_desc_lo(sV + s * L::kKVBytes, L::kKVBytes);
+#pragma unroll 4
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            mma_bf16_ts(d_tmem, a_tmem + kk * 8, desc_join(v_lo + kk * (16 * L::kRowBytes / 16), kDescHi), idesc_o,
+                        (!first || kk > 0) ? 1u : 0u);
+          tc_commit(&bars[L::kBarODone + w]);
+        };
+        // Per key tile j the order is S0(j+1), P0 V(j), S1(j+1), P1 V(j): each
+        // warpgroup's next score tile and its P V follow its own progress, so
+        // neither warpgroup's MMAs queue behind the other's softmax.
+        for (int u = u_begin; u < p.n_units && ok; u += u_step, ++uc) {
+          // first score tiles of the unit
+          ok = mbar_wait(&bars[L::kBarQFull], uc & 1, wc);
+          if (ok) ok = mbar_wait(&bars[L::kBarKFull + kc % L::kKVStages], (kc / L::kKVStages) & 1, wc);
+          for (int w = 0; w < kQTiles && ok; ++w) {
+            if (gs > 0 && !(ok = mbar_wait(&bars[L::kBarSFree + w], (gs - 1) & 1, wc))) break;
+            tc_fence_after_sync();
+            issue_s(w, kc % L::kKVStages);
+          }
+          if (!ok) break;
+          tc_commit(&bars[L::kBarKEmpty + kc % L::kKVStages]);
+          if (nt == 1) tc_commit(&bars[L::kBarQEmpty]);
+          ++kc;
+          ++gs;
+          for (int j = 0; j < nt && ok; ++j) {
+            const bool has_next = j + 1 < nt;
+            const int sk = kc % L::kKVStages;
+            const int sv = vc % L::kKVStages;
+            if (has_next) ok = mbar_wait(&bars[L::kBarKFull + sk], (kc / L::kKVStages) & 1, wc);
+            if (ok) ok = mbar_wait(&bars[L::kBarVFull + sv], (vc / L::kKVStages) & 1, wc);
+            for (int w = 0; w < kQTiles && ok; ++w) {
+              if (has_next) {
+                if (!(ok = mbar_wait(&bars[L::kBarSFree + w], (gs - 1) & 1, wc))) break;
+                tc_fence_after_sync();
+                issue_s(w, sk);
+              }
+              if (!(ok = mbar_wait(&bars[L::kBarPFull + w], gp & 1, wc))) break;
+              // the first P V of a unit overwrites O: the epilogue of the
+              // previous unit must have read it
+              if (j == 0 && uc > 0 && !(ok = mbar_wait(&bars[L::kBarOFree + w], (uc - 1) & 1, wc))) break;
+              tc_fence_after_sync();
+              issue_pv(w, sv, j == 0);
+            }
+            if (!ok) break;
+            if (has_next) {
+              tc_commit(&bars[L::kBarKEmpty + sk]);
+              // after the unit's last score MMAs the Q slot can be refilled
+              if (j + 2 == nt) tc_commit(&bars[L::kBarQEmpty]);
+              ++kc;
+              ++gs;
+            }
+            tc_commit(&bars[L::kBarVEmpty + sv]);
+            ++vc;
+            ++gp;
+          }
+        }
+        // Every MMA issued above completes before Tensor Memory is released.
+        tc_commit(&bars[L::kBarDrain]);
+        mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
+      }
+    } else {
+      // ============================================================== key-mask warp
+      // Lane l owns keys 4l..4l+3 of each tile; the mask bytes of tile j+1 are
+      // loaded while tile j is processed.  For the untransposed bias tile the
+      // warp writes one mask word per key pair beside the bias slot and the
+      // softmax warps apply it while unpacking the bias; for the transposed
+      // tile (one key per 256-byte row) it writes -inf over the masked rows.
+      // Without a key mask and with whole key tiles the softmax warps wait on
+      // the TMA barrier directly and this warp has nothing to do.
+      bool ok = kBiasT ? (p.needs_mask != 0) : kMasked;
+      int gt = 0;  // key tiles processed (all units)
+      for (int u = u_begin; u < p.n_units && ok; u += u_step) {
+        const Unit un = decode_unit(p, u);
+        const uint8_t *mrow = p.mask ? p.mask + (int64_t)un.b * p.mask_sb : nullptr;
+        auto load_word = [&](int j) -> uint32_t {  // byte e nonzero = key 4*lane+e takes part
+          const int key0 = j * kBN + 4 * lane;
+          if (mrow == nullptr) return 0x01010101u;
+          if (p.mask_vec4 && key0 + 3 < p.Nk) return __ldg(reinterpret_cast<const uint32_t *>(mrow + key0));
+          uint32_t wv = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (key0 + e < p.Nk) wv |= uint32_t(__ldg(mrow + (int64_t)(key0 + e) * p.mask_sk) != 0) << (8 * e);
+          return wv;
+        };
+        uint32_t next_word = load_word(0);
+        for (int j = 0; j < nt && ok; ++j, ++gt) {
+          const uint32_t word = next_word;
+          if (j + 1 < nt) next_word = load_word(j + 1);
+          const int key0 = j * kBN + 4 * lane;
+          uint32_t inv = 0;  // bit e: key 4*lane + e of the tile is masked or past the end
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (key0 + e >= p.Nk || ((word >> (8 * e)) & 0xFFu) == 0) inv |= 1u << e;
+          // keep-masks of the key pairs (4l, 4l+1) and (4l+2, 4l+3)
+          const uint2 keep = make_uint2(((inv & 1u) ? 0u : 0x0000FFFFu) | ((inv & 2u) ? 0u : 0xFFFF0000u),
+                                        ((inv & 4u) ? 0u : 0x0000FFFFu) | ((inv & 8u) ? 0u : 0xFFFF0000u));
+          const uint32_t any = kBiasT ? __ballot_sync(0xffffffffu, inv != 0) : 0u;
+          const int t = gt % kBiasStages;
+          for (int w = 0; w < kQTiles && ok; ++w) {
+            const int slot = w * kBiasStages + t;
+            ok = mbar_wait(&bars[L::kBarBiasFull + slot], (gt / kBiasStages) & 1, wc);
+            if (!ok) break;
+            if (!kBiasT) {
+              reinterpret_cast<uint2 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[lane] = keep;
+            } else if (any) {
+              uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
+              uint32_t rem = any;
+              while (rem) {
+                const int src = __ffs(rem) - 1;
+                rem &= rem - 1;
+                uint32_t bits = __shfl_sync(0xffffffffu, inv, src);
+                while (bits) {
+                  const int e = __ffs(bits) - 1;
+                  bits &= bits - 1;
+                  // row 4*src+e of the [key][query] tile: 128 bf16 = 256 bytes
+                  reinterpret_cast<uint2 *>(tile + (4 * src + e) * 256)[lane] =
+                      make_uint2(0xFF80FF80u, 0xFF80FF80u);
+                }
+              }
+              fence_proxy_async_smem();
+            }
+            __syncwarp();
+            mbar_arrive(&bars[L::kBarBiasReady + slot]);
+          }
+        }
       }
     }
-  }
   } else {
     // ================================================================ softmax warpgroups
     setmaxnreg_inc<kRegsSoftmax>();
@@ -419,122 +480,126 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
     const uint32_t tP = tmem + lane_base + 256 + w * 64;
     const uint32_t tO = tmem + lane_base + 384 + w * 64;
     const float tau = p.tau;
-    float m_cur = -INFINITY;   // maximum used for P and l
-    float m_true = -INFINITY;  // true running maximum
-    float l = 0.f;
+    const bool relay = kBiasT ? (p.needs_mask != 0) : kMasked;
     bool ok = true;
-    for (int j = 0; j < nt && ok; ++j) {
-      ok = mbar_wait(&bars[L::kBarSFull + w], j & 1, wc);
-      if (!ok) break;
-      tc_fence_after_sync();
-      uint32_t sreg[kBN];
-#pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sreg[c * 32]));
-      tmem_wait_ld();
-      tc_fence_before_sync();
-      mbar_arrive(&bars[L::kBarSFree + w]);
-
-      const int slot = w * kBiasStages + (j % kBiasStages);
-      const bool relay = kBiasT ? (p.needs_mask != 0) : kMasked;
-      ok = mbar_wait(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (j / kBiasStages) & 1, wc);
-      if (!ok) break;
-      const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
-      // x = tau * s + bias, two keys per packed fma
-      float2 x[kBN / 2];
-      const float2 tau2 = make_float2(tau, tau);
-      if (kBiasT) {
-        const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
-#pragma unroll
-        for (int c = 0; c < kBN; c += 2) {
-          const float2 bv = make_float2(__uint_as_float(uint32_t(col[c * kBM]) << 16),
-                                        __uint_as_float(uint32_t(col[(c + 1) * kBM]) << 16));
-          x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2, bv);
-        }
-      } else {
-#pragma unroll
-        for (int c8 = 0; c8 < kBN / 8; ++c8) {
-          const int box = c8 >> 3, chunk = c8 & 7;
-          const uint4 bv = *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 +
-                                                            ((chunk ^ (t & 7)) << 4));
-          uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
-          if (kMasked) {
-            // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
-            const uint4 kv = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
-            const uint32_t keep[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) wv[e] = (wv[e] & keep[e]) | (~keep[e] & 0xFF80FF80u);
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = c8 * 8 + 2 * e;
-            x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2,
-                             make_float2(bf16lo_to_f32(wv[e]), bf16hi_to_f32(wv[e])));
-          }
-        }
-      }
-      mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
-
-      // tile maximum: eight independent chains
-      float m8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(x[i].x, x[i].y);
-#pragma unroll
-      for (int i = 8; i < kBN / 2; ++i) m8[i & 7] = max3f(m8[i & 7], x[i].x, x[i].y);
-      const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      m_true = fmaxf(m_true, mx);
-      const bool need = mx > m_cur + kRescaleThreshold;
-      float alpha = 1.f;
-      if (need) {
-        alpha = (m_cur == -INFINITY) ? 0.f : ex2_approx((m_cur - mx) * kLog2e);
-        l *= alpha;
-        m_cur = mx;
-      }
-      const float neg_m = (m_cur == -INFINITY) ? 0.f : -m_cur * kLog2e;
-      const float2 l2e2 = make_float2(kLog2e, kLog2e), negm2 = make_float2(neg_m, neg_m);
-      uint32_t pk[kBN / 2];
-      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int i = 0; i < kBN / 2; ++i) {
-        const float2 a = ffma2(x[i], l2e2, negm2);
-        // every kExpEmuEvery-th key pair takes the software exp2 on the FMA pipe
-        const float2 pv = (kExpEmuEvery > 0 && i % kExpEmuEvery == kExpEmuEvery - 1)
-                              ? exp2_poly2(a)
-                              : make_float2(ex2_approx(a.x), ex2_approx(a.y));
-        ls[i & 3] = fadd2(ls[i & 3], pv);
-        pk[i] = pack_bf16x2(pv.x, pv.y);
-      }
-      const float2 lsum2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
-      l += lsum2.x + lsum2.y;
-
-      if (j > 0) {
-        ok = mbar_wait(&bars[L::kBarODone + w], (j - 1) & 1, wc);
+    int gt = 0;  // key tiles processed (all units)
+    for (int u = u_begin; u < p.n_units && ok; u += u_step) {
+      float m_cur = -INFINITY;   // maximum used for P and l
+      float m_true = -INFINITY;  // true running maximum
+      float l = 0.f;
+      for (int j = 0; j < nt && ok; ++j, ++gt) {
+        ok = mbar_wait(&bars[L::kBarSFull + w], gt & 1, wc);
         if (!ok) break;
         tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, need)) {
-          // rescale this warp's rows of O (lanes without a new maximum use 1)
+        uint32_t sreg[kBN];
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c, o);
-            tmem_wait_ld();
+        for (int c = 0; c < kBN / 32; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sreg[c * 32]));
+        tmem_wait_ld();
+        tc_fence_before_sync();
+        mbar_arrive(&bars[L::kBarSFree + w]);
+
+        const int slot = w * kBiasStages + (gt % kBiasStages);
+        ok = mbar_wait(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1, wc);
+        if (!ok) break;
+        const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
+        // x = tau * s + bias, two keys per packed fma
+        float2 x[kBN / 2];
+        const float2 tau2 = make_float2(tau, tau);
+        if (kBiasT) {
+          const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + c, o);
+          for (int c = 0; c < kBN; c += 2) {
+            const float2 bv = make_float2(__uint_as_float(uint32_t(col[c * kBM]) << 16),
+                                          __uint_as_float(uint32_t(col[(c + 1) * kBM]) << 16));
+            x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2, bv);
+          }
+        } else {
+#pragma unroll
+          for (int c8 = 0; c8 < kBN / 8; ++c8) {
+            const int box = c8 >> 3, chunk = c8 & 7;
+            const uint4 bv = *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 +
+                                                              ((chunk ^ (t & 7)) << 4));
+            uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
+            if (kMasked) {
+              // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
+              const uint4 kv = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
+              const uint32_t keep[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) wv[e] = (wv[e] & keep[e]) | (~keep[e] & 0xFF80FF80u);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = c8 * 8 + 2 * e;
+              x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2,
+                               make_float2(bf16lo_to_f32(wv[e]), bf16hi_to_f32(wv[e])));
+            }
           }
         }
-      }
-#pragma unroll
-      for (int c = 0; c < kBN / 2; c += 32) tmem_st32(tP + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
-      tmem_wait_st();
-      tc_fence_before_sync();
-      mbar_arrive(&bars[L::kBarPFull + w]);
-    }
+        mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
 
-    // ---------------------------------------------------------------- epilogue
-    if (ok) ok = mbar_wait(&bars[L::kBarODone + w], (nt - 1) & 1, wc);
-    if (ok) {
+        // tile maximum: eight independent chains
+        float m8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(x[i].x, x[i].y);
+#pragma unroll
+        for (int i = 8; i < kBN / 2; ++i) m8[i & 7] = max3f(m8[i & 7], x[i].x, x[i].y);
+        const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        m_true = fmaxf(m_true, mx);
+        const bool need = mx > m_cur + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = (m_cur == -INFINITY) ? 0.f : ex2_approx((m_cur - mx) * kLog2e);
+          l *= alpha;
+          m_cur = mx;
+        }
+        const float neg_m = (m_cur == -INFINITY) ? 0.f : -m_cur * kLog2e;
+        const float2 l2e2 = make_float2(kLog2e, kLog2e), negm2 = make_float2(neg_m, neg_m);
+        uint32_t pk[kBN / 2];
+        float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int i = 0; i < kBN / 2; ++i) {
+          const float2 a = ffma2(x[i], l2e2, negm2);
+          // every kExpEmuEvery-th key pair takes the software exp2 on the FMA pipe
+          const float2 pv = (kExpEmuEvery > 0 && i % kExpEmuEvery == kExpEmuEvery - 1)
+                                ? exp2_poly2(a)
+                                : make_float2(ex2_approx(a.x), ex2_approx(a.y));
+          ls[i & 3] = fadd2(ls[i & 3], pv);
+          pk[i] = pack_bf16x2(pv.x, pv.y);
+        }
+        const float2 lsum2 = fadd2(fadd2(ls[0], ls[1]), fadd2(ls[2], ls[3]));
+        l += lsum2.x + lsum2.y;
+
+        // P(j) overwrites the P buffer that P V(j-1) read, possibly the last
+        // one of the previous unit
+        if (gt > 0) {
+          ok = mbar_wait(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
+          if (!ok) break;
+          tc_fence_after_sync();
+          if (j > 0 && __any_sync(0xffffffffu, need)) {
+            // rescale this warp's rows of O (lanes without a new maximum use 1)
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(tO + c, o);
+            }
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < kBN / 2; c += 32) tmem_st32(tP + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(&bars[L::kBarPFull + w]);
+      }
+
+      // -------------------------------------------------------------- epilogue
+      if (ok) ok = mbar_wait(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
+      if (!ok) break;
       tc_fence_after_sync();
-      const int row = q0 + w * kBM + t;
       float o[D];
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -544,16 +609,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[c + e] = __uint_as_float(r[e]);
       }
+      // O is in registers: the next unit's first P V may overwrite it
+      tc_fence_before_sync();
+      mbar_arrive(&bars[L::kBarOFree + w]);
+      const Unit un = decode_unit(p, u);  // derived here so it is not live across the tile loop
+      const int row = un.q0 + w * kBM + t;
+      const int b = un.b, h = un.h;
       if (row < p.Nq) {
         const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
         if (kEpi == kEpiForward) {
           float g[D];
           if (kGate) {
-            const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + b * p.gate_sb + h * p.gate_sh +
-                                                              (int64_t)row * p.gate_sn);
+            const uint4 *gptr = reinterpret_cast<const uint4 *>(p.gate + b * p.gate_sb + h * p.gate_sh +
+                                                                (int64_t)row * p.gate_sn);
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {
-              const uint4 gv = gp[c];
+              const uint4 gv = gptr[c];
               const uint32_t wv[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {

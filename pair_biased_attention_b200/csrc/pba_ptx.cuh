@@ -204,6 +204,26 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)swizzle_mode << 61);
 }
 
+// The same descriptor split into its two 32-bit halves, so a loop over K steps
+// only adds to the address field of the low half.
+__device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo_bytes, uint32_t swizzle_mode) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (swizzle_mode << 29);
+}
+__device__ __forceinline__ uint64_t desc_join(uint32_t lo, uint32_t hi) { return (uint64_t(hi) << 32) | lo; }
+// Descriptor of the low half lo + add, formed right where it is used (the
+// volatile asm keeps the compiler from computing every descriptor of an
+// unrolled loop up front, which costs the issuing thread its registers).
+__device__ __forceinline__ uint64_t desc_at(uint32_t lo, uint32_t add, uint32_t hi) {
+  uint64_t d;
+  asm volatile("{\n\t.reg .b32 t;\n\tadd.u32 t, %1, %2;\n\tmov.b64 %0, {t, %3};\n\t}"
+               : "=l"(d)
+               : "r"(lo), "r"(add), "r"(hi));
+  return d;
+}
+
 // TMEM loads/stores of the 32x32b shape: thread t of the warp reads/writes
 // lane (base lane + t), N consecutive 32-bit columns.
 #define PBA_R8(b) "=r"(r[b + 0]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), \
