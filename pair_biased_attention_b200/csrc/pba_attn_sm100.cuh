@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           const int t = gt % kBiasStages;
           for (int w = 0; w < kQTiles && ok; ++w) {
             const int slot = w * kBiasStages + t;
-            ok = mbar_wait(&bars[L::kBarBiasFull + slot], (gt / kBiasStages) & 1, wc);
+            ok = mbar_wait<false>(&bars[L::kBarBiasFull + slot], (gt / kBiasStages) & 1, wc);
             if (!ok) break;
             if (!kBiasT) {
               reinterpret_cast<uint2 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[lane] = keep;
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       float m_true = -INFINITY;  // true running maximum
       float l = 0.f;
       for (int j = 0; j < nt && ok; ++j, ++gt) {
-        ok = mbar_wait(&bars[L::kBarSFull + w], gt & 1, wc);
+        ok = mbar_wait<false>(&bars[L::kBarSFull + w], gt & 1, wc);
         if (!ok) break;
         tc_fence_after_sync();
         uint32_t sreg[kBN];
@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         mbar_arrive(&bars[L::kBarSFree + w]);
 
         const int slot = w * kBiasStages + (gt % kBiasStages);
-        ok = mbar_wait(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1, wc);
+        ok = mbar_wait<false>(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1, wc);
         if (!ok) break;
         const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
         // x = tau * s + bias, two keys per packed fma
@@ -573,7 +573,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         // P(j) overwrites the P buffer that P V(j-1) read, possibly the last
         // one of the previous unit
         if (gt > 0) {
-          ok = mbar_wait(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
+          ok = mbar_wait<false>(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
           if (!ok) break;
           tc_fence_after_sync();
           if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       }
 
       // -------------------------------------------------------------- epilogue
-      if (ok) ok = mbar_wait(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
+      if (ok) ok = mbar_wait<false>(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
       if (!ok) break;
       tc_fence_after_sync();
       float o[D];

@@ -83,6 +83,15 @@ struct WaitCtl {
   uint64_t timeout_ns;
 };
 
+// Waits for the phase of `bar` with the given parity.  Returns false when the
+// time limit runs out (after raising the abort word and recording
+// kErrTimeout) or, with kPollAbort, as soon as another thread has raised the
+// abort word.  Waits of a full warp whose lanes must leave together (the
+// collective Tensor Memory accesses and shuffles after them need every lane)
+// pass kPollAbort = false: all lanes then end on the same condition, the
+// phase or their own time limit, never on a flag one lane saw set and
+// another did not.  Clean-up waits after an abort use it as well.
+template <bool kPollAbort = true>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const WaitCtl &w) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -91,7 +100,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     if (PBA_WAIT_HINT_NS ? mbar_try_wait_hint(bar, parity, PBA_WAIT_HINT_NS) : mbar_try_wait(bar, parity))
       return true;
     if ((++iter & 3u) == 0) {
-      if (*w.abort_flag) return false;
+      if (kPollAbort && *w.abort_flag) return false;
       if (global_timer_ns() - t0 > w.timeout_ns) {
         *w.abort_flag = 1;
         atomicCAS(w.err, 0, kErrTimeout);

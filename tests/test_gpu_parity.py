@@ -210,6 +210,26 @@ def test_shapes(cuda_device, Nq, Nk, D, mask_frac, dtype):
     assert np.abs(mp[fin] - ref["m"][fin]).max(initial=0) <= LSE_TOL
 
 
+@pytest.mark.parametrize("D", [32, 64])
+@pytest.mark.parametrize("scale", [0.125, 0.25, 0.13, 0.3])
+def test_bias_modes(cuda_device, D, scale):
+    """A softmax scale that is a power of two has the tensor core add the bias
+    (scores S = Q K^T + bias / scale, the mask as a rank-1 MMA); any other
+    scale has the softmax warps add it.  Both against the oracle, masked and
+    ragged, forward and partial."""
+    q, k, v, bias, mask = W.random_attn(2, 3, 333, 421, D, seed=int(scale * 1000) + D, device=cuda_device,
+                                        mask_frac=0.1)
+    out, lse = pba.pba_forward(q, k, v, bias, mask, softmax_scale=scale)
+    ref = oracle.pba(q, k, v, bias, mask, softmax_scale=scale)
+    _cmp(f"bias mode D={D} scale={scale}", out, lse, ref)
+    o_p, m_p, l_p = pba.pba_partial(q, k, v, bias, mask, softmax_scale=scale)
+    _cmp(f"bias mode partial D={D} scale={scale}", o_p, m_p + torch.log(l_p), ref)
+    # unmasked whole tiles: no mask MMA
+    q, k, v, bias, _ = W.random_attn(1, 2, 256, 512, D, seed=D + 1, device=cuda_device)
+    out, lse = pba.pba_forward(q, k, v, bias, softmax_scale=scale)
+    _cmp(f"bias mode unmasked D={D} scale={scale}", out, lse, oracle.pba(q, k, v, bias, softmax_scale=scale))
+
+
 def test_bias_broadcast_over_heads_and_batch(cuda_device):
     q, k, v, bias, mask = W.random_attn(2, 4, 200, 300, 64, seed=5, device=cuda_device, mask_frac=0.1)
     b1 = bias[:1, :1]  # [1,1,Nq,Nk] -> strides 0 over b and h
@@ -226,17 +246,24 @@ def _padded_clone(b):
     return full[..., :nk]
 
 
-def test_minus_inf_bias_and_fully_masked_rows(cuda_device):
-    q, k, v, bias, _ = W.random_attn(1, 2, 300, 260, 64, seed=9, device=cuda_device)
+@pytest.mark.parametrize("D,scale", [(64, None), (32, 0.25), (32, None), (64, 0.1)])
+def test_minus_inf_bias_and_fully_masked_rows(cuda_device, D, scale):
+    """-inf bias entries exclude their keys.  With a power-of-two scale the
+    first pass (bias added by the tensor core) turns them into NaN rows, and
+    the re-run recomputes those units; the result must not show it."""
+    q, k, v, bias, mask = W.random_attn(1, 2, 600, 260, D, seed=9, device=cuda_device, mask_frac=0.05)
     bias = _padded_clone(bias)
     bias[0, 0, 5, :] = -math.inf              # row with no valid key
     bias[0, 1, 7, ::3] = -math.inf            # scattered -inf entries
     bias[0, 1, 200:260, :130] = -math.inf     # a whole tile region
-    out, lse = pba.pba_forward(q, k, v, bias)
-    ref = oracle.pba(q, k, v, bias)
+    out, lse = pba.pba_forward(q, k, v, bias, mask, softmax_scale=scale)
+    ref = oracle.pba(q, k, v, bias, mask, softmax_scale=scale)
     _cmp("minus inf bias", out, lse, ref)
     assert torch.all(out[0, 0, 5] == 0) and lse[0, 0, 5].item() == -math.inf
     assert not torch.isnan(out.float()).any()
+    o_p, m_p, l_p = pba.pba_partial(q, k, v, bias, mask, softmax_scale=scale)
+    _cmp("minus inf bias, partial", o_p, m_p + torch.log(l_p), ref)
+    assert not torch.isnan(o_p).any() and not torch.isnan(l_p).any()
 
 
 def test_empty_inputs(cuda_device):
