@@ -61,6 +61,8 @@ def _lib(mutant: int = 0):
             lib.oracle_merge.restype = ctypes.c_int
             lib.oracle_tri_attn_lines.argtypes = [_i64, _i64, _i64, ctypes.c_int, _dbl, _i64] + [_p] * 8 + [ctypes.c_int]
             lib.oracle_tri_attn_lines.restype = ctypes.c_int
+            lib.oracle_tri_proj.argtypes = [_i64] * 4 + [_p] * 5 + [ctypes.c_int]
+            lib.oracle_tri_proj.restype = ctypes.c_int
             lib.oracle_threads_used.argtypes = [ctypes.c_int]
             lib.oracle_threads_used.restype = ctypes.c_int
             _LIBS[mutant] = lib
@@ -203,3 +205,21 @@ def tri_attn(q, k, v, bias, g=None, pair_mask=None, ending: bool = False, lines=
         pm = _u8(pair_mask)
         ml = pm[:, idx].T if ending else pm[idx]
     return tri_attn_lines(sl(q), sl(k), sl(v), bias, sl(g), ml, ending, softmax_scale, nthreads, mutant)
+
+
+def tri_proj(z, w, wb, rows=None, nthreads: int = 0, mutant: int = 0):
+    """Triangle projections in fp64: z [N,N,c] (or [R,c]), w [c,F] (the
+    q | k | v | g column blocks), wb [c,H].  ``rows`` selects flat pair rows
+    r = i*N + j (None = all).  Returns out [R,F] and bias [H,R] for the
+    selected rows."""
+    c = z.shape[-1]
+    zf = _f64(z).reshape(-1, c)
+    if rows is not None:
+        zf = np.ascontiguousarray(zf[np.asarray(rows, dtype=np.int64)])
+    wf, wbf = _f64(w), _f64(wb)
+    R, F, H = zf.shape[0], wf.shape[1], wbf.shape[1]
+    out = np.zeros((R, F))
+    bias = np.zeros((H, R))
+    rc = _lib(mutant).oracle_tri_proj(R, c, F, H, _ptr(zf), _ptr(wf), _ptr(wbf), _ptr(out), _ptr(bias), nthreads)
+    assert rc == 0
+    return {"out": out, "bias": bias}

@@ -365,3 +365,53 @@ int oracle_tri_attn_lines(int64_t N, int64_t H, int64_t D, int ending, double ta
   parallel_rows(tri_row, &c, nl * N * H, 2 * N + D, nthreads);
   return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Triangle projections (Fold-CP, Figure 2(a): the pair tensor z gives  */
+/* the queries, keys, values, gate and the per-head bias of triangle     */
+/* attention).  For every pair row r = (i, j) of z [N*N][c]:            */
+/*   out[r][f] = sum_c z[r][c] * w[c][f]     f < F (w [c][F])           */
+/*   bias[h][r] = sum_c z[r][c] * wb[c][h]   h < H (wb [c][H])           */
+/* i.e. q|k|v|g are the column blocks of out, and the bias is laid out   */
+/* [H][N][N].  Plain fp64 dot products, one pair row per call.           */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  int64_t c, F, H;
+  const double *z, *w, *wb;
+  double *out, *bias;
+  int64_t rows;
+} proj_ctx;
+
+static void proj_row(const void *vctx, int64_t r, double *scratch) {
+  (void)scratch;
+  const proj_ctx *x = (const proj_ctx *)vctx;
+  const double *zr = x->z + r * x->c;
+  for (int64_t f = 0; f < x->F; ++f) {
+    double acc = 0.0;
+    for (int64_t cc = 0; cc < x->c; ++cc)
+#if ORACLE_MUTANT == 10 /* planted: weight read transposed */
+      acc += zr[cc] * x->w[(f % x->c) * x->F + (cc % x->F)];
+#else
+      acc += zr[cc] * x->w[cc * x->F + f];
+#endif
+    x->out[r * x->F + f] = acc;
+  }
+  for (int64_t h = 0; h < x->H; ++h) {
+    double acc = 0.0;
+    for (int64_t cc = 0; cc < x->c; ++cc)
+#if ORACLE_MUTANT == 11 /* planted: bias taken from the first weight columns */
+      acc += zr[cc] * x->w[cc * x->F + h];
+#else
+      acc += zr[cc] * x->wb[cc * x->H + h];
+#endif
+    x->bias[h * x->rows + r] = acc;
+  }
+}
+
+int oracle_tri_proj(int64_t rows, int64_t c, int64_t F, int64_t H, const double *z, const double *w,
+                    const double *wb, double *out, double *bias, int nthreads) {
+  if (rows < 0 || c < 1 || F < 0 || H < 0) return 1;
+  proj_ctx x = {c, F, H, z, w, wb, out, bias, rows};
+  parallel_rows(proj_row, &x, rows, 1, nthreads);
+  return 0;
+}

@@ -350,6 +350,52 @@ def test_golden_triangle(case, gate):
     assert np.abs(en["lse"].transpose(1, 0, 2) - np.array(case["ending_lse"])).max() < 1e-14
 
 
+# ---------------------------------------------------------------- triangle projections
+# Fold-CP, Figure 2(a): q, k, v, g and the per-head bias of triangle attention
+# are linear maps of the pair tensor z; the oracle writes them out as fp64 dot
+# products.  Pinned against numpy's matmul (an independent implementation),
+# closed forms and linearity.
+def _proj_problem(N=6, c=16, F=24, H=3, seed=0):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((N, N, c)), rng.standard_normal((c, F)), rng.standard_normal((c, H))
+
+
+def test_proj_matches_numpy_matmul():
+    z, w, wb = _proj_problem()
+    r = oracle.tri_proj(z, w, wb)
+    zf = z.reshape(-1, z.shape[-1])
+    assert np.abs(r["out"] - zf @ w).max() < 1e-12
+    assert np.abs(r["bias"] - (zf @ wb).T).max() < 1e-12
+    assert r["bias"].shape == (3, 36)  # [H, N*N]: b[h, i, j] at h*N*N + i*N + j
+
+
+def test_proj_one_hot_rows_select_weight_rows():
+    _, w, wb = _proj_problem(c=16, F=24, H=3)
+    z = np.eye(16)[[3, 0, 15, 7]]  # pair rows that pick weight rows 3, 0, 15, 7
+    r = oracle.tri_proj(z, w, wb)
+    assert np.array_equal(r["out"], w[[3, 0, 15, 7]])
+    assert np.array_equal(r["bias"], wb[[3, 0, 15, 7]].T)
+
+
+def test_proj_hand_worked_example():
+    # z = [1, 2]; W = [[1, 0, 2], [3, 1, 0]]; W_b = [[1], [-1]]
+    # out = [1*1 + 2*3, 1*0 + 2*1, 1*2 + 2*0] = [7, 2, 2]; bias = 1 - 2 = -1
+    r = oracle.tri_proj(np.array([[1.0, 2.0]]), np.array([[1.0, 0, 2], [3, 1, 0]]), np.array([[1.0], [-1.0]]))
+    assert np.array_equal(r["out"], [[7.0, 2.0, 2.0]]) and np.array_equal(r["bias"], [[-1.0]])
+
+
+def test_proj_linearity_and_row_selection():
+    z1, w, wb = _proj_problem(seed=1)
+    z2, _, _ = _proj_problem(seed=2)
+    a, b = 0.75, -2.5
+    r = oracle.tri_proj(a * z1 + b * z2, w, wb)
+    r1, r2 = oracle.tri_proj(z1, w, wb), oracle.tri_proj(z2, w, wb)
+    assert np.abs(r["out"] - (a * r1["out"] + b * r2["out"])).max() < 1e-12
+    rows = [35, 0, 17]
+    rs = oracle.tri_proj(z1, w, wb, rows=rows)
+    assert np.array_equal(rs["out"], r1["out"][rows]) and np.array_equal(rs["bias"], r1["bias"][:, rows])
+
+
 # ---------------------------------------------------------------- planted mistakes
 def _pin_suite(mutant):
     """Run a compact set of the pins against an oracle build; return the
@@ -390,6 +436,11 @@ def _pin_suite(mutant):
     keep = (~empty).numpy()
     if np.abs(r["o"][keep] - o_ref.numpy()[keep]).max() > 1e-10:
         fails += 1
+    z, w, wb = _proj_problem(seed=3)
+    pr = oracle.tri_proj(z, w, wb, mutant=mutant)
+    zf = z.reshape(-1, z.shape[-1])
+    if np.abs(pr["out"] - zf @ w).max() > 1e-12 or np.abs(pr["bias"] - (zf @ wb).T).max() > 1e-12:
+        fails += 1
     return fails
 
 
@@ -397,6 +448,6 @@ def test_default_build_passes_compact_pins():
     assert _pin_suite(0) == 0
 
 
-@pytest.mark.parametrize("mutant", range(1, 10))
+@pytest.mark.parametrize("mutant", range(1, 12))
 def test_planted_mistake_is_caught(mutant):
     assert _pin_suite(mutant) > 0, f"planted mistake {mutant} went unnoticed"

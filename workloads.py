@@ -147,12 +147,10 @@ def block_order(cfg: AttnConfig) -> list[int]:
     return torch.randperm(cfg.blocks, generator=g).tolist()
 
 
-def tri_inputs(cfg: TriConfig, device="cpu"):
-    """q, k, v, g [N,N,H,D] bf16 and bias [H,N,N] bf16 from a seeded pair tensor.
-
-    z [N,N,c] ~ N(0,1) and W_q, W_k, W_v, W_g [c, H*D], W_b [c, H] ~ N(0, 1/c),
-    all rounded to bf16; each projection is z W taken in fp32 and rounded to
-    bf16.  The bias is laid out [H, N, N] with b[h, j, k] from pair (j, k)."""
+def tri_pair_inputs(cfg: TriConfig, device="cpu"):
+    """The seeded draws of a triangle workload: z [N,N,c] ~ N(0,1) and the
+    weights W_q | W_k | W_v | W_g as one [c, 4*H*D] matrix and W_b [c, H],
+    ~ N(0, 1/c), all rounded to bf16."""
     dev = torch.device(device)
     gen = torch.Generator(dev.type).manual_seed(cfg.seed)
     N, c, H, D = cfg.N, cfg.c, cfg.H, cfg.D
@@ -160,10 +158,22 @@ def tri_inputs(cfg: TriConfig, device="cpu"):
     wstd = 1.0 / math.sqrt(c)
     ws = [(torch.randn((c, H * D), generator=gen, device=dev) * wstd).to(torch.bfloat16) for _ in range(4)]
     wb = (torch.randn((c, H), generator=gen, device=dev) * wstd).to(torch.bfloat16)
-    zf = z.float().reshape(N * N, c)
+    return z, torch.cat(ws, dim=1).contiguous(), wb
+
+
+def tri_inputs(cfg: TriConfig, device="cpu"):
+    """q, k, v, g [N,N,H,D] bf16 and bias [H,N,N] bf16 from a seeded pair tensor.
+
+    The draws of tri_pair_inputs; each projection is z W taken in fp32 and
+    rounded to bf16 (input synthesis for the attention, which takes the bf16
+    tensors as given).  The bias is laid out [H, N, N] with b[h, j, k] from
+    pair (j, k)."""
+    N, H, D = cfg.N, cfg.H, cfg.D
+    z, w, wb = tri_pair_inputs(cfg, device)
+    zf = z.float().reshape(N * N, cfg.c)
     outs = []
-    for w in ws:
-        outs.append((zf @ w.float()).to(torch.bfloat16).reshape(N, N, H, D).contiguous())
+    for i in range(4):
+        outs.append((zf @ w[:, i * H * D:(i + 1) * H * D].float()).to(torch.bfloat16).reshape(N, N, H, D).contiguous())
     bias = (zf @ wb.float()).to(torch.bfloat16).reshape(N, N, H).permute(2, 0, 1).contiguous()
     q, k, v, g = outs
     return q, k, v, g, bias
