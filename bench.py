@@ -271,7 +271,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["none", "pba4k", "tri512"], default="none",
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024"], default="none",
                     help="run one small case only (for ncu captures); prints no JSON line")
     args = ap.parse_args()
     world, rank, local, pg = dist_setup(args)
@@ -362,6 +362,7 @@ def main():
         "clocks": clk,
     }
 
+    line["tri_proj"] = run_proj(args, pba, tcfg, dev, stream, pg, peaks)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -375,6 +376,39 @@ def main():
 
         dist.destroy_process_group()
     return 0
+
+
+def run_proj(args, pba, tcfg, dev, stream, pg, peaks):
+    """The triangle projections of the triangle workload (tri_proj_forward:
+    z [N,N,c] -> q, k, v, g [N,N,H,D] and bias [H,N,N]), timed on their own
+    after the step: K calls after 3 warm-up calls, CUDA events on the stream.
+    HBM-bound: algorithmic bytes = z read once + the five outputs written."""
+    z, w, wb = W.tri_pair_inputs(tcfg, dev)
+    N2 = tcfg.N * tcfg.N
+    outs = tuple(torch.empty((tcfg.N, tcfg.N, tcfg.H, tcfg.D), dtype=torch.bfloat16, device=dev) for _ in range(4))
+    pb = torch.empty((tcfg.H, tcfg.N, tcfg.N), dtype=torch.bfloat16, device=dev)
+    call = lambda: pba.tri_proj_forward(z, w, wb, tcfg.H, out=outs, bias=pb, stream=stream)
+    for _ in range(3):
+        call()
+    barrier(pg)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        call()
+    e.record(stream)
+    barrier(pg)
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("the projection kernel recorded a device error")
+    ms = max_over_ranks(s.elapsed_time(e), pg) / args.steps
+    nbytes = N2 * tcfg.c * 2 + 4 * N2 * tcfg.H * tcfg.D * 2 + tcfg.H * N2 * 2
+    flops = 2.0 * N2 * tcfg.c * (4 * tcfg.H * tcfg.D + tcfg.H)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"ms_per_call": ms, "calls": args.steps, "gpu_launches": args.steps,
+            "workload": f"tri{tcfg.N}: z [{tcfg.N},{tcfg.N},{tcfg.c}] bf16 -> q,k,v,g [N,N,{tcfg.H},{tcfg.D}] + bias [{tcfg.H},N,N]",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
+                         "kernel": "pba_proj_sm100_kernel (tri_proj_forward)", "peak_source": peaks["source"],
+                         "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
 
 
 def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops):
@@ -417,7 +451,11 @@ def run_profile_case(args, pba, dev):
     """One small case for ncu: pba4k = pba_forward at N=4096 (bias 512 MB,
     larger than L2) after one warm-up launch; tri512 = triangle attention
     N=512 both orientations."""
-    if args.profile == "pba4k":
+    if args.profile == "proj1024":
+        z, w, wb = W.tri_pair_inputs(W.TRI1024, dev)
+        for _ in range(2):
+            pba.tri_proj_forward(z, w, wb, W.TRI1024.H)
+    elif args.profile == "pba4k":
         cfg = W.AttnConfig("pba4k", B=1, N=4096, H=16, D=64, dtype=torch.bfloat16, seed=4, mask="random5")
         q, k, v, bias, mask = W.attn_inputs(cfg, dev)
         for _ in range(2):

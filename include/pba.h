@@ -171,6 +171,29 @@ PBA_API pba_status tri_attn_forward(int64_t N, int64_t H, int64_t D, int32_t ori
                             const void *k, const void *v, const void *bias, const void *gate,
                             const uint8_t *pair_mask, void *out, float *lse, void *stream);
 
+/*
+ * tri_proj_forward -- the triangle projections of a pair tensor in one pass
+ * (Fold-CP, Figure 2(a): triangle attention draws its queries, keys, values,
+ * gate and per-head bias from the pair representation).
+ *   z       [N][N][c]   bf16, device; pair row r = i*N + j, c in {64, 128}
+ *   w_qkvg  [c][4*H*D]  bf16, device; column blocks W_q | W_k | W_v | W_g
+ *   w_b     [c][H]      bf16, device
+ * For every pair row r, in fp32 sums of the bf16 products, rounded once to bf16:
+ *   q[r][:] = z[r] W_q,  k[r][:] = z[r] W_k,  v[r][:] = z[r] W_v,  g[r][:] = z[r] W_g
+ *     (q, k, v, g [N][N][H][D] bf16, device: the layout tri_attn_forward takes;
+ *      g is the gate before its sigmoid)
+ *   bias[h][i][j] = z[i*N+j] W_b[:, h]   (bias [H][N][N] bf16, device)
+ * Requires H*D = 128, H in {1, 2, 4, 8}, N <= 32768.  z, w_qkvg, q, k, v, g
+ * must be 16-byte aligned, w_b and bias 2-byte aligned (else
+ * PBA_ERR_INVALID_ARG); other shapes give PBA_ERR_UNSUPPORTED.  N = 0 does
+ * nothing and accepts NULL buffers.  The caller
+ * owns every buffer; nothing is allocated.  Asynchronous on `stream`.
+ * The pages fix no layout for these maps; q|k|v|g as column blocks of one
+ * weight is the plain reading of "projections of the pair representation".
+ */
+PBA_API pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const void *z, const void *w_qkvg,
+                                    const void *w_b, void *q, void *k, void *v, void *g, void *bias, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 PBA_API const char *pba_status_string(pba_status status);
 

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "PbaError", "PBA_OK", "PBA_ERR_INVALID_ARG", "PBA_ERR_UNSUPPORTED", "PBA_ERR_CUDA", "PBA_ERR_TIMEOUT",
-    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward",
+    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward",
     "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_selftest_exp2",
     "pba_status_string",
 ]
@@ -81,6 +81,8 @@ def load_library() -> ctypes.CDLL:
     lib.tri_attn_forward.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
                                      _p, _p, _p, _p, _p, _p, _p, _p, _p]
     lib.tri_attn_forward.restype = st
+    lib.tri_proj_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 9
+    lib.tri_proj_forward.restype = st
     lib.pba_status_string.argtypes = [st]
     lib.pba_status_string.restype = ctypes.c_char_p
     lib.pba_last_device_error.argtypes = [_p]
@@ -276,6 +278,34 @@ def tri_attn_forward(q, k, v, bias, gate=None, pair_mask=None, orientation="star
                                                                _ptr(pair_mask), _ptr(out), _ptr(lse),
                                                                _stream(stream)))
     return out, lse
+
+
+def tri_proj_forward(z, w_qkvg, w_b, H, out=None, bias=None, stream=None):
+    """Triangle projections of a pair tensor, bf16.  z [N,N,c] (contiguous),
+    w_qkvg [c, 4*H*D] (column blocks W_q | W_k | W_v | W_g), w_b [c, H].
+    Returns q, k, v, g [N,N,H,D] and bias [H,N,N]; ``out`` may pass the four
+    output tensors."""
+    for n, t in (("z", z), ("w_qkvg", w_qkvg), ("w_b", w_b)):
+        _cuda(n, t, torch.bfloat16)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    N, N2, c = z.shape
+    if N2 != N or w_qkvg.shape[0] != c or w_b.shape != (c, H) or w_qkvg.shape[1] % (4 * H) != 0:
+        raise ValueError("z must be [N,N,c], w_qkvg [c, 4*H*D], w_b [c,H]")
+    D = w_qkvg.shape[1] // (4 * H)
+    if out is None:
+        out = tuple(torch.empty((N, N, H, D), dtype=torch.bfloat16, device=z.device) for _ in range(4))
+    if bias is None:
+        bias = torch.empty((H, N, N), dtype=torch.bfloat16, device=z.device)
+    for n, t in zip(("q", "k", "v", "g", "bias"), tuple(out) + (bias,)):
+        _cuda(n, t, torch.bfloat16)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    q, k, v, g = out
+    _check("tri_proj_forward", load_library().tri_proj_forward(N, c, H, D, _ptr(z), _ptr(w_qkvg), _ptr(w_b), _ptr(q),
+                                                               _ptr(k), _ptr(v), _ptr(g), _ptr(bias),
+                                                               _stream(stream)))
+    return q, k, v, g, bias
 
 
 def pba_last_device_error(stream=None) -> int:

@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -13,6 +14,7 @@
 
 #include "pba.h"
 #include "pba_attn_sm100.cuh"
+#include "pba_proj_sm100.cuh"
 #include "pba_simt.cuh"
 
 // Device error word: written by kernels whose bounded waits ran out, read and
@@ -366,6 +368,20 @@ pba_status attn_common(const pba_attn_desc *d, const void *q, const void *k, con
   return run_tc(t, stream);
 }
 
+// ------------------------------------------------------------ triangle projections
+template <int kH>
+cudaError_t launch_proj(const pba::ProjParams &p, int grid, cudaStream_t stream) {
+  auto kern = pba::pba_proj_sm100_kernel<kH>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pba::ProjLayout::kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, pba::kProjThreads, pba::ProjLayout::kSmemAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
@@ -466,6 +482,66 @@ pba_status tri_attn_forward(int64_t N, int64_t H, int64_t D, int32_t orient, flo
   t.lse_s[2] = ending ? N * H : H;
   t.gate = gate;
   return run_tc(t, static_cast<cudaStream_t>(stream_ptr));
+}
+
+pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const void *z, const void *w_qkvg,
+                            const void *w_b, void *q, void *k, void *v, void *g, void *bias, void *stream_ptr) {
+  if (N < 0 || N > 32768 || H < 1 || D < 1) return PBA_ERR_INVALID_ARG;
+  if ((c != 64 && c != 128) || H * D != 128 || (H != 1 && H != 2 && H != 4 && H != 8)) return PBA_ERR_UNSUPPORTED;
+  if (N == 0) return PBA_OK;  // nothing to read or write; zero-extent buffers may be NULL
+  if (z == nullptr || w_qkvg == nullptr || w_b == nullptr || q == nullptr || k == nullptr || v == nullptr ||
+      g == nullptr || bias == nullptr)
+    return PBA_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(w_qkvg) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) ||
+      (reinterpret_cast<uintptr_t>(w_b) & 1u) || (reinterpret_cast<uintptr_t>(bias) & 1u))
+    return PBA_ERR_INVALID_ARG;
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  const int64_t rows = N * N;
+  pba::ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  {
+    const uint64_t dims[4] = {uint64_t(c), uint64_t(rows), 1, 1};
+    const int64_t st[3] = {c * 2, 0, 0};
+    const uint32_t box[4] = {64, uint32_t(pba::kProjRows), 1, 1};
+    if (!make_map(&p.tm_z, z, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(pba::kProjCols), uint64_t(c), 1, 1};
+    const int64_t st[3] = {int64_t(pba::kProjCols) * 2, 0, 0};
+    const uint32_t box[4] = {64, uint32_t(c), 1, 1};
+    if (!make_map(&p.tm_w, w_qkvg, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+  }
+  for (int m = 0; m < 4; ++m) {
+    void *const dst[4] = {q, k, v, g};
+    const uint64_t dims[4] = {uint64_t(pba::kProjCols / 4), uint64_t(rows), 1, 1};
+    const int64_t st[3] = {int64_t(pba::kProjCols / 4) * 2, 0, 0};
+    const uint32_t box[4] = {32, uint32_t(pba::kProjRows), 1, 1};
+    if (!make_map(&p.tm_out[m], dst[m], dims, st, box, CU_TENSOR_MAP_SWIZZLE_64B)) return PBA_ERR_INVALID_ARG;
+  }
+  p.rows = rows;
+  p.c = int(c);
+  p.n_tiles = int((rows + pba::kProjRows - 1) / pba::kProjRows);
+  p.wb = static_cast<const uint16_t *>(w_b);
+  p.out[0] = static_cast<uint16_t *>(q);
+  p.out[1] = static_cast<uint16_t *>(k);
+  p.out[2] = static_cast<uint16_t *>(v);
+  p.out[3] = static_cast<uint16_t *>(g);
+  p.bias = static_cast<uint16_t *>(bias);
+  p.err = device_error_word();
+  if (p.err == nullptr) return PBA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return PBA_ERR_CUDA;
+  const int grid = std::min(p.n_tiles, sms);
+  cudaStream_t st = static_cast<cudaStream_t>(stream_ptr);
+  cudaError_t e = H == 1   ? launch_proj<1>(p, grid, st)
+                  : H == 2 ? launch_proj<2>(p, grid, st)
+                  : H == 4 ? launch_proj<4>(p, grid, st)
+                           : launch_proj<8>(p, grid, st);
+  return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
 }
 
 const char *pba_status_string(pba_status status) {

@@ -28,7 +28,7 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "pba_status_string",
+    for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pba_status_string",
               "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout",
               "pba_selftest_exp2"):
         assert n in names
@@ -139,6 +139,28 @@ def test_tri_rejects_unaligned_pointer(lib):
     unaligned = ctypes.c_void_p(0x10008)
     assert lib.tri_attn_forward(16, 4, 32, 0, 0.0, unaligned, FAKE, FAKE, FAKE, None, None, FAKE, None,
                                 None) == pba.PBA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("N,c,H,D,expect", [
+    (16, 96, 4, 32, pba.PBA_ERR_UNSUPPORTED),    # c not 64 or 128
+    (16, 128, 4, 16, pba.PBA_ERR_UNSUPPORTED),   # H*D != 128
+    (16, 128, 3, 32, pba.PBA_ERR_UNSUPPORTED),   # H not a power of two up to 8
+    (-1, 128, 4, 32, pba.PBA_ERR_INVALID_ARG),
+    (40000, 128, 4, 32, pba.PBA_ERR_INVALID_ARG),  # N*N row coordinates past int32
+])
+def test_proj_rejects_bad_shapes(lib, N, c, H, D, expect):
+    assert lib.tri_proj_forward(N, c, H, D, *([FAKE] * 8), None) == expect
+
+
+def test_proj_rejects_null_and_unaligned(lib):
+    args = [FAKE] * 8
+    for i in range(8):
+        bad = list(args)
+        bad[i] = None
+        assert lib.tri_proj_forward(16, 128, 4, 32, *bad, None) == pba.PBA_ERR_INVALID_ARG
+    bad = list(args)
+    bad[0] = ctypes.c_void_p(0x10008)  # z not 16-byte aligned
+    assert lib.tri_proj_forward(16, 128, 4, 32, *bad, None) == pba.PBA_ERR_INVALID_ARG
 
 
 def test_selftest_rejects_bad_limit(lib):
