@@ -488,6 +488,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       float m_true = -INFINITY;  // true running maximum
       float l = 0.f;
       for (int j = 0; j < nt && ok; ++j, ++gt) {
+        // The bias tile lands long before it is used: wait for it first and
+        // start loading its first half from shared memory, so that those loads
+        // overlap the wait for the score tile and its Tensor Memory load.
+        const int slot = w * kBiasStages + (gt % kBiasStages);
+        ok = mbar_wait<false>(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1, wc);
+        if (!ok) break;
+        const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
+        constexpr int kPre = kBN / 16;  // 8-key groups loaded ahead
+        uint4 bpre[kPre];                // untransposed tile: 8 bf16 per group
+        uint32_t tpre[kBiasT ? 4 * kPre : 1];  // transposed tile: 1 bf16 per key
+        if (kBiasT) {
+          const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
+#pragma unroll
+          for (int c = 0; c < 4 * kPre; ++c) tpre[c] = col[c * kBM];
+        } else {
+#pragma unroll
+          for (int c8 = 0; c8 < kPre; ++c8)
+            bpre[c8] = *reinterpret_cast<const uint4 *>(tile + t * 128 + ((c8 ^ (t & 7)) << 4));
+        }
+
         ok = mbar_wait<false>(&bars[L::kBarSFull + w], gt & 1, wc);
         if (!ok) break;
         tc_fence_after_sync();
@@ -499,10 +519,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         tc_fence_before_sync();
         mbar_arrive(&bars[L::kBarSFree + w]);
 
-        const int slot = w * kBiasStages + (gt % kBiasStages);
-        ok = mbar_wait<false>(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1, wc);
-        if (!ok) break;
-        const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
         // x = tau * s + bias, two keys per packed fma
         float2 x[kBN / 2];
         const float2 tau2 = make_float2(tau, tau);
@@ -510,16 +526,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
 #pragma unroll
           for (int c = 0; c < kBN; c += 2) {
-            const float2 bv = make_float2(__uint_as_float(uint32_t(col[c * kBM]) << 16),
-                                          __uint_as_float(uint32_t(col[(c + 1) * kBM]) << 16));
+            const uint32_t b0 = c < 4 * kPre ? tpre[c] : uint32_t(col[c * kBM]);
+            const uint32_t b1 = c + 1 < 4 * kPre ? tpre[c + 1] : uint32_t(col[(c + 1) * kBM]);
+            const float2 bv = make_float2(__uint_as_float(b0 << 16), __uint_as_float(b1 << 16));
             x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2, bv);
           }
         } else {
 #pragma unroll
           for (int c8 = 0; c8 < kBN / 8; ++c8) {
             const int box = c8 >> 3, chunk = c8 & 7;
-            const uint4 bv = *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 +
-                                                              ((chunk ^ (t & 7)) << 4));
+            const uint4 bv = c8 < kPre ? bpre[c8]
+                                       : *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 +
+                                                                          ((chunk ^ (t & 7)) << 4));
             uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
             if (kMasked) {
               // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
