@@ -63,6 +63,8 @@ def _lib(mutant: int = 0):
             lib.oracle_tri_attn_lines.restype = ctypes.c_int
             lib.oracle_tri_proj.argtypes = [_i64] * 4 + [_p] * 5 + [ctypes.c_int]
             lib.oracle_tri_proj.restype = ctypes.c_int
+            lib.oracle_pwa.argtypes = [_i64] * 4 + [_p] * 6 + [ctypes.c_int]
+            lib.oracle_pwa.restype = ctypes.c_int
             lib.oracle_threads_used.argtypes = [ctypes.c_int]
             lib.oracle_threads_used.restype = ctypes.c_int
             _LIBS[mutant] = lib
@@ -223,3 +225,16 @@ def tri_proj(z, w, wb, rows=None, nthreads: int = 0, mutant: int = 0):
     rc = _lib(mutant).oracle_tri_proj(R, c, F, H, _ptr(zf), _ptr(wf), _ptr(wbf), _ptr(out), _ptr(bias), nthreads)
     assert rc == 0
     return {"out": out, "bias": bias}
+
+
+def pwa(v, bias, key_mask=None, g=None, nthreads: int = 0, mutant: int = 0):
+    """Pair weighted averaging in fp64 (the reading stated in pba_oracle.c):
+    v [S,N,H,D], bias [H,N,N], key_mask [N] or None, g [S,N,H,D] or None.
+    Returns out [S,N,H,D] and lse [H,N]."""
+    vf, bf, gf, mk = _f64(v), _f64(bias), _f64(g), _u8(key_mask)
+    S, N, H, D = vf.shape
+    out = np.zeros((S, N, H, D))
+    lse = np.zeros((H, N))
+    rc = _lib(mutant).oracle_pwa(S, N, H, D, _ptr(vf), _ptr(bf), _ptr(gf), _ptr(mk), _ptr(out), _ptr(lse), nthreads)
+    assert rc == 0
+    return {"o": out, "lse": lse}

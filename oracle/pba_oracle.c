@@ -415,3 +415,66 @@ int oracle_tri_proj(int64_t rows, int64_t c, int64_t F, int64_t H, const double 
   parallel_rows(proj_row, &x, rows, 1, nthreads);
   return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Pair weighted averaging (Fold-CP, Table 1 row "Pair Weighted Avg.": */
+/* serial time B*H*S*N^2*D, distributed as a "2D ring + tiled softmax", */
+/* and Figure 2: it shares the softmax-merge archetype of the ring      */
+/* attention).  The pages give no formula; the reading used here is a   */
+/* softmax over the pair-bias logits alone, shared by the S sequences:  */
+/*   w[h][i][j] = exp(b[h][i][j] - m) / l  over valid keys j            */
+/*     (m = max, l = sum of exp(b - m) over valid j of row (h, i))      */
+/*   o[s][i][h][:] = sum_j w[h][i][j] v[s][j][h][:]                      */
+/*   out = o * sigmoid(g) when a gate is given; lse[h][i] = m + ln l.   */
+/* v, g, out [S][N][H][D]; bias [H][N][N]; key mask [N] or NULL.        */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  int64_t S, N, H, D;
+  const double *v, *bias, *g;
+  const uint8_t *mask;
+  double *out, *lse;
+} pwa_ctx;
+
+static void pwa_row(const void *vctx, int64_t row, double *w) {
+  const pwa_ctx *x = (const pwa_ctx *)vctx;
+  const int64_t h = row / x->N, i = row % x->N, N = x->N, H = x->H, D = x->D;
+  const double *brow = x->bias + (h * N + i) * N;
+  double m = -INFINITY, l = 0.0;
+  for (int64_t j = 0; j < N; ++j) {
+    int valid = (x->mask == NULL || x->mask[j] != 0) && brow[j] != -INFINITY;
+#if ORACLE_MUTANT == 12 /* planted: key mask ignored */
+    valid = brow[j] != -INFINITY;
+#endif
+    w[j] = valid ? brow[j] : -INFINITY;
+    if (w[j] > m) m = w[j];
+  }
+  if (m != -INFINITY)
+    for (int64_t j = 0; j < N; ++j) {
+      w[j] = (w[j] == -INFINITY) ? 0.0 : exp(w[j] - m);
+      l += w[j];
+    }
+  for (int64_t s = 0; s < x->S; ++s) {
+    for (int64_t d = 0; d < D; ++d) {
+      double acc = 0.0;
+      if (l > 0.0)
+        for (int64_t j = 0; j < N; ++j)
+#if ORACLE_MUTANT == 13 /* planted: values of sequence 0 for every sequence */
+          acc += w[j] * x->v[((0 * N + j) * H + h) * D + d];
+#else
+          acc += w[j] * x->v[((s * N + j) * H + h) * D + d];
+#endif
+      const double o = (l > 0.0) ? acc / l : 0.0;
+      const int64_t at = ((s * N + i) * H + h) * D + d;
+      x->out[at] = x->g ? o * sigmoid(x->g[at]) : o;
+    }
+  }
+  if (x->lse) x->lse[h * N + i] = (l > 0.0) ? m + log(l) : -INFINITY;
+}
+
+int oracle_pwa(int64_t S, int64_t N, int64_t H, int64_t D, const double *v, const double *bias, const double *g,
+               const uint8_t *mask, double *out, double *lse, int nthreads) {
+  if (S < 0 || N < 0 || H < 1 || D < 1) return 1;
+  pwa_ctx x = {S, N, H, D, v, bias, g, mask, out, lse};
+  parallel_rows(pwa_row, &x, H * N, N, nthreads);
+  return 0;
+}

@@ -396,6 +396,65 @@ def test_proj_linearity_and_row_selection():
     assert np.array_equal(rs["out"], r1["out"][rows]) and np.array_equal(rs["bias"], r1["bias"][:, rows])
 
 
+# ---------------------------------------------------------------- pair weighted averaging
+# Fold-CP, Table 1 row "Pair Weighted Avg." (B*H*S*N^2*D; "2D ring + tiled
+# softmax") and Figure 2 (shares the softmax-merge archetype).  Reading: a
+# softmax over the pair-bias logits alone, shared by the S sequences.  Pinned
+# against pair-biased attention with zero queries (a different oracle path),
+# torch's fp64 softmax and einsum, and closed forms.
+def _pwa_problem(S=3, N=11, H=2, D=4, seed=0, mask_frac=0.3, neg_inf_frac=0.0):
+    g = torch.Generator().manual_seed(seed)
+    v = torch.randn((S, N, H, D), generator=g, dtype=torch.float64)
+    bias = torch.randn((H, N, N), generator=g, dtype=torch.float64) * 2
+    if neg_inf_frac:
+        bias[torch.rand((H, N, N), generator=g) < neg_inf_frac] = -math.inf
+    mask = (torch.rand((N,), generator=g) >= mask_frac).to(torch.uint8)
+    gate = torch.randn((S, N, H, D), generator=g, dtype=torch.float64)
+    return v, bias, mask, gate
+
+
+def test_pwa_is_attention_with_zero_queries():
+    v, bias, mask, _ = _pwa_problem(neg_inf_frac=0.1)
+    r = oracle.pwa(v, bias, mask)
+    S, N, H, D = v.shape
+    q = torch.zeros((S, H, N, D), dtype=torch.float64)
+    vt = v.permute(0, 2, 1, 3).contiguous()             # [S,H,N,D]
+    bt = bias[None].expand(S, H, N, N).contiguous()      # the same logits for every sequence
+    a = oracle.pba(q, q, vt, bt, mask[None].expand(S, N).contiguous())
+    assert np.abs(r["o"] - a["o"].transpose(0, 2, 1, 3)).max() < 1e-13
+    fin = np.isfinite(r["lse"])
+    assert np.array_equal(fin, np.isfinite(a["lse"][0]))
+    assert np.abs(r["lse"][fin] - a["lse"][0][fin]).max() < 1e-13
+
+
+def test_pwa_matches_torch_softmax_einsum_with_gate():
+    v, bias, mask, gate = _pwa_problem(S=4, N=17, H=3, D=5, seed=1)
+    r = oracle.pwa(v, bias, mask, gate)
+    logits = bias.masked_fill(mask[None, None, :] == 0, -math.inf)
+    w = torch.softmax(logits, dim=-1)                    # [H,N,N]
+    o = torch.einsum("hij,sjhd->sihd", w, v) * torch.sigmoid(gate)
+    assert np.abs(r["o"] - o.numpy()).max() < 1e-13
+    assert np.abs(r["lse"] - torch.logsumexp(logits, dim=-1).numpy()).max() < 1e-13
+
+
+def test_pwa_closed_forms():
+    v, _, mask, _ = _pwa_problem(S=2, N=9, H=2, D=3, seed=2, mask_frac=0.4)
+    # equal logits: the mean of the valid values
+    r = oracle.pwa(v, torch.zeros((2, 9, 9), dtype=torch.float64), mask)
+    valid = mask.bool()
+    assert np.abs(r["o"] - v[:, valid].mean(dim=1, keepdim=True).expand_as(v).numpy()).max() < 1e-14
+    assert np.allclose(r["lse"], math.log(int(valid.sum())))
+    # one finite logit per row: exactly that key's values
+    pick = torch.tensor([4, 0, 8, 2, 2, 7, 1, 3, 5])
+    bias = torch.full((2, 9, 9), -math.inf, dtype=torch.float64)
+    bias[:, torch.arange(9), pick] = 1.5
+    r = oracle.pwa(v, bias, None)
+    assert np.array_equal(r["o"], v[:, pick].numpy()) and np.allclose(r["lse"], 1.5)
+    # no valid key: zeros and -inf
+    r = oracle.pwa(v, bias, torch.zeros(9, dtype=torch.uint8))
+    assert np.all(r["o"] == 0) and np.all(r["lse"] == -np.inf)
+
+
 # ---------------------------------------------------------------- planted mistakes
 def _pin_suite(mutant):
     """Run a compact set of the pins against an oracle build; return the
@@ -441,6 +500,12 @@ def _pin_suite(mutant):
     zf = z.reshape(-1, z.shape[-1])
     if np.abs(pr["out"] - zf @ w).max() > 1e-12 or np.abs(pr["bias"] - (zf @ wb).T).max() > 1e-12:
         fails += 1
+    v, bias, mask, _ = _pwa_problem(seed=4)
+    pw = oracle.pwa(v, bias, mask, mutant=mutant)
+    logits = bias.masked_fill(mask[None, None, :] == 0, -math.inf)
+    o = torch.einsum("hij,sjhd->sihd", torch.softmax(logits, dim=-1), v)
+    if np.abs(pw["o"] - o.numpy()).max() > 1e-12:
+        fails += 1
     return fails
 
 
@@ -448,6 +513,6 @@ def test_default_build_passes_compact_pins():
     assert _pin_suite(0) == 0
 
 
-@pytest.mark.parametrize("mutant", range(1, 12))
+@pytest.mark.parametrize("mutant", range(1, 14))
 def test_planted_mistake_is_caught(mutant):
     assert _pin_suite(mutant) > 0, f"planted mistake {mutant} went unnoticed"

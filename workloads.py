@@ -22,6 +22,9 @@ benchmark inputs for this path, so every tensor here is synthetic:
   large16k  N=16384, H=16, D=64, bf16, bias ~ N(0,1) (8.6 GB); a random key
             mask of round(0.05 N) = 819 keys (seed 4).
   tri1024   as tri512 with N=1024 (seed 5).
+  pwa512    pair weighted averaging, S=16 sequences, N=512, H=8, D=32; v,
+            gate, bias ~ N(0,1) bf16, last 5% of keys masked (seed 6).
+  pwa4k     as pwa512 with S=64, N=4096 (seed 7).
 
 "N(0, 2)" and "N(0, 1/c)" are read as (mean, variance).
 
@@ -177,6 +180,38 @@ def tri_inputs(cfg: TriConfig, device="cpu"):
     bias = (zf @ wb.float()).to(torch.bfloat16).reshape(N, N, H).permute(2, 0, 1).contiguous()
     q, k, v, g = outs
     return q, k, v, g, bias
+
+
+@dataclass(frozen=True)
+class PwaConfig:
+    """Pair weighted averaging: S sequences of N tokens, H heads of D values,
+    one bias [H,N,N] shared by the sequences."""
+    name: str
+    S: int
+    N: int
+    H: int
+    D: int
+    seed: int
+    pad_frac: float = 0.0  # last round(pad_frac*N) keys masked (padding)
+
+
+PWA512 = PwaConfig("pwa512", S=16, N=512, H=8, D=32, seed=6, pad_frac=0.05)
+PWA4K = PwaConfig("pwa4k", S=64, N=4096, H=8, D=32, seed=7, pad_frac=0.05)
+
+
+def pwa_inputs(cfg: PwaConfig, device="cpu"):
+    """v, gate [S,N,H,D] ~ N(0,1), bias [H,N,N] ~ N(0,1), all bf16, and a key
+    padding mask [N] uint8 (or None), drawn in that order from one seed."""
+    dev = torch.device(device)
+    gen = torch.Generator(dev.type).manual_seed(cfg.seed)
+    v = torch.randn((cfg.S, cfg.N, cfg.H, cfg.D), generator=gen, device=dev).to(torch.bfloat16)
+    bias = torch.randn((cfg.H, cfg.N, cfg.N), generator=gen, device=dev).to(torch.bfloat16)
+    gate = torch.randn((cfg.S, cfg.N, cfg.H, cfg.D), generator=gen, device=dev).to(torch.bfloat16)
+    mask = None
+    if cfg.pad_frac:
+        mask = torch.ones((cfg.N,), dtype=torch.uint8, device=dev)
+        mask[cfg.N - int(round(cfg.pad_frac * cfg.N)):] = 0
+    return v, bias, mask, gate
 
 
 def sample_rows(N: int, count: int, seed: int, tile: int = 128) -> list[int]:
