@@ -271,7 +271,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024"], default="none",
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "pwa4k"], default="none",
                     help="run one small case only (for ncu captures); prints no JSON line")
     args = ap.parse_args()
     world, rank, local, pg = dist_setup(args)
@@ -363,6 +363,7 @@ def main():
     }
 
     line["tri_proj"] = run_proj(args, pba, tcfg, dev, stream, pg, peaks)
+    line["pwa"] = run_pwa(args, pba, dev, stream, pg, peaks, clk)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -411,6 +412,43 @@ def run_proj(args, pba, tcfg, dev, stream, pg, peaks):
                          "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
 
 
+def run_pwa(args, pba, dev, stream, pg, peaks, clk):
+    """Pair weighted averaging on pwa4k (S=64 sequences, N=4096, H=8, D=32,
+    gate, 5% key padding), timed on its own after the step: K calls after 3
+    warm-up calls, CUDA events on the stream.  Compute-bound: 2*H*S*N^2*D
+    FLOPs on the tensor cores and H*N^2 exps per 192-feature tile on the
+    exp2 unit (16 per clock per SM)."""
+    cfg = W.PWA4K
+    v, bias, mask, gate = W.pwa_inputs(cfg, dev)
+    out = torch.empty_like(v)
+    lse = torch.empty((cfg.H, cfg.N), dtype=torch.float32, device=dev)
+    call = lambda: pba.pwa_forward(v, bias, mask, gate, out, lse, stream=stream)
+    for _ in range(3):
+        call()
+    barrier(pg)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        call()
+    e.record(stream)
+    barrier(pg)
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("the pair weighted averaging kernel recorded a device error")
+    ms = max_over_ranks(s.elapsed_time(e), pg) / args.steps
+    flops = 2.0 * cfg.H * cfg.S * cfg.N * cfg.N * cfg.D
+    ftiles = -(-cfg.S // (192 // cfg.D))
+    exps = cfg.H * cfg.N * cfg.N * ftiles
+    tflops = flops / (ms / 1e3) / 1e12
+    sm_hz = (clk.get("sm_mhz") or 1965.0) * 1e6 if isinstance(clk, dict) else 1965e6
+    exp_floor_ms = exps / (16 * torch.cuda.get_device_properties(dev).multi_processor_count * sm_hz) * 1e3
+    return {"ms_per_call": ms, "calls": args.steps, "gpu_launches": args.steps, "tflops": tflops,
+            "workload": f"pwa4k: S={cfg.S} N={cfg.N} H={cfg.H} D={cfg.D}, gate, 5% key padding, bias [H,N,N]",
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "kernel": "pba_pwa_sm100_kernel (pwa_forward)",
+                         "peak_source": peaks["source"], "exp2_floor_ms": exp_floor_ms,
+                         "exp2_frac": exp_floor_ms / ms}}
+
+
 def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops):
     """Same metric through the public call with the inputs starting in pinned
     host memory and the outputs read back each step."""
@@ -451,7 +489,11 @@ def run_profile_case(args, pba, dev):
     """One small case for ncu: pba4k = pba_forward at N=4096 (bias 512 MB,
     larger than L2) after one warm-up launch; tri512 = triangle attention
     N=512 both orientations."""
-    if args.profile == "proj1024":
+    if args.profile == "pwa4k":
+        v, bias, mask, gate = W.pwa_inputs(W.PWA4K, dev)
+        for _ in range(2):
+            pba.pwa_forward(v, bias, mask, gate)
+    elif args.profile == "proj1024":
         z, w, wb = W.tri_pair_inputs(W.TRI1024, dev)
         for _ in range(2):
             pba.tri_proj_forward(z, w, wb, W.TRI1024.H)

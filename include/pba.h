@@ -194,6 +194,26 @@ PBA_API pba_status tri_attn_forward(int64_t N, int64_t H, int64_t D, int32_t ori
 PBA_API pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const void *z, const void *w_qkvg,
                                     const void *w_b, void *q, void *k, void *v, void *g, void *bias, void *stream);
 
+/*
+ * pwa_forward -- pair weighted averaging (Fold-CP, Table 1 row "Pair
+ * Weighted Avg.", serial time B*H*S*N^2*D, distributed as a "2D ring + tiled
+ * softmax"; Figure 2: it shares the softmax-merge archetype of the ring
+ * attention).  The pages print no formula; the reading implemented here is a
+ * softmax over the pair-bias logits alone, shared by the S sequences:
+ *   w[h][i][:]    = softmax_j( bias[h][i][j] )  over keys j with key_mask[j] != 0
+ *   o[s][i][h][:] = sum_j w[h][i][j] v[s][j][h][:]
+ *   out = o * sigmoid(gate) (gate NULL: out = o);  lse[h][i] = natural log-sum-exp
+ *   v, gate, out [S][N][H][D] bf16, device; bias [H][N][N] bf16, device;
+ *   key_mask [N] uint8, device, or NULL; lse [H][N] float, device, or NULL.
+ * A row with no valid key gives out = 0 and lse = -inf.  D in {32, 64}
+ * (else PBA_ERR_UNSUPPORTED); N a multiple of 8 and v, bias, gate, out
+ * 16-byte aligned (else PBA_ERR_INVALID_ARG).  S = 0 or N = 0 writes nothing
+ * and accepts NULL buffers.  The caller owns every buffer; nothing is
+ * allocated.  Asynchronous on `stream`.
+ */
+PBA_API pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v, const void *bias,
+                               const uint8_t *key_mask, const void *gate, void *out, float *lse, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 PBA_API const char *pba_status_string(pba_status status);
 

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "PbaError", "PBA_OK", "PBA_ERR_INVALID_ARG", "PBA_ERR_UNSUPPORTED", "PBA_ERR_CUDA", "PBA_ERR_TIMEOUT",
-    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward",
+    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pwa_forward",
     "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_selftest_exp2",
     "pba_status_string",
 ]
@@ -83,6 +83,8 @@ def load_library() -> ctypes.CDLL:
     lib.tri_attn_forward.restype = st
     lib.tri_proj_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 9
     lib.tri_proj_forward.restype = st
+    lib.pwa_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 7
+    lib.pwa_forward.restype = st
     lib.pba_status_string.argtypes = [st]
     lib.pba_status_string.restype = ctypes.c_char_p
     lib.pba_last_device_error.argtypes = [_p]
@@ -306,6 +308,30 @@ def tri_proj_forward(z, w_qkvg, w_b, H, out=None, bias=None, stream=None):
                                                                _ptr(k), _ptr(v), _ptr(g), _ptr(bias),
                                                                _stream(stream)))
     return q, k, v, g, bias
+
+
+def pwa_forward(v, bias, key_mask=None, gate=None, out=None, lse=None, return_lse=True, stream=None):
+    """Pair weighted averaging, bf16: v, gate [S,N,H,D] (contiguous), bias
+    [H,N,N], key_mask [N] uint8 or None.  Returns out [S,N,H,D] and lse [H,N]."""
+    for n, t in (("v", v), ("bias", bias), ("gate", gate)):
+        _cuda(n, t, torch.bfloat16)
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _cuda("key_mask", key_mask, torch.uint8)
+    S, N, H, D = v.shape
+    if tuple(bias.shape) != (H, N, N) or (gate is not None and gate.shape != v.shape):
+        raise ValueError("bias must be [H,N,N] and gate [S,N,H,D]")
+    if key_mask is not None and (tuple(key_mask.shape) != (N,) or not key_mask.is_contiguous()):
+        raise ValueError("key_mask must be a contiguous [N] uint8 tensor")
+    if out is None:
+        out = torch.empty_like(v)
+    if lse is None and return_lse:
+        lse = torch.empty((H, N), dtype=torch.float32, device=v.device)
+    _cuda("out", out, torch.bfloat16)
+    _cuda("lse", lse, torch.float32)
+    _check("pwa_forward", load_library().pwa_forward(S, N, H, D, _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
+                                                     _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def pba_last_device_error(stream=None) -> int:

@@ -15,6 +15,7 @@
 #include "pba.h"
 #include "pba_attn_sm100.cuh"
 #include "pba_proj_sm100.cuh"
+#include "pba_pwa_sm100.cuh"
 #include "pba_simt.cuh"
 
 // Device error word: written by kernels whose bounded waits ran out, read and
@@ -382,6 +383,32 @@ cudaError_t launch_proj(const pba::ProjParams &p, int grid, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ pair weighted averaging
+template <int D, bool kGate, bool kMasked>
+cudaError_t launch_pwa(const pba::PwaParams &p, int grid, cudaStream_t stream) {
+  using L = pba::PwaLayout<D>;
+  auto kern = pba::pba_pwa_sm100_kernel<D, kGate, kMasked>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+        fa.numRegs * pba::kAttnThreads < pba::kRegSplitTotal)
+      attr_err = cudaErrorInvalidConfiguration;
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, pba::kAttnThreads, L::kSmemAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_pwa(const pba::PwaParams &p, int grid, bool gate, cudaStream_t st) {
+  const bool m = p.masked != 0;
+  if (gate) return m ? launch_pwa<D, true, true>(p, grid, st) : launch_pwa<D, true, false>(p, grid, st);
+  return m ? launch_pwa<D, false, true>(p, grid, st) : launch_pwa<D, false, false>(p, grid, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -541,6 +568,63 @@ pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const vo
                   : H == 2 ? launch_proj<2>(p, grid, st)
                   : H == 4 ? launch_proj<4>(p, grid, st)
                            : launch_proj<8>(p, grid, st);
+  return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v, const void *bias,
+                       const uint8_t *key_mask, const void *gate, void *out, float *lse, void *stream_ptr) {
+  if (S < 0 || N < 0 || H < 1 || S > 65535 || N > 65535 || H > 4096) return PBA_ERR_INVALID_ARG;
+  if (D != 32 && D != 64) return PBA_ERR_UNSUPPORTED;
+  if (N % 8 != 0) return PBA_ERR_INVALID_ARG;  // bias rows are tile rows: 16-byte strides
+  if (S == 0 || N == 0) return PBA_OK;        // nothing to write; zero-extent buffers may be NULL
+  if (v == nullptr || bias == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(bias) || !aligned16(out) || (gate != nullptr && !aligned16(gate)))
+    return PBA_ERR_INVALID_ARG;
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  const int slabs = 192 / int(D);
+  pba::PwaParams p;
+  std::memset(&p, 0, sizeof(p));
+  {
+    // v [S][N][H][D] as (D, N, H, S)
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(N), uint64_t(H), uint64_t(S)};
+    const int64_t st[3] = {H * D * 2, D * 2, N * H * D * 2};
+    const uint32_t box[4] = {uint32_t(D), uint32_t(pba::kBN), 1, uint32_t(slabs)};
+    if (!make_map(&p.tm_v, v, dims, st, box, D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+      return PBA_ERR_INVALID_ARG;
+  }
+  {
+    // bias [H][N][N] as (keys, rows, H, 1): two 64-key boxes per tile
+    const uint64_t dims[4] = {uint64_t(N), uint64_t(N), uint64_t(H), 1};
+    const int64_t st[3] = {N * 2, N * N * 2, 0};
+    const uint32_t box[4] = {64, uint32_t(pba::kBM), 1, 1};
+    if (!make_map(&p.tm_bias, bias, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+  }
+  p.S = int(S);
+  p.N = int(N);
+  p.H = int(H);
+  p.n_qblocks = int((N + pba::kQTiles * pba::kBM - 1) / (pba::kQTiles * pba::kBM));
+  p.n_ftiles = int((S + slabs - 1) / slabs);
+  const int64_t n_units = int64_t(H) * p.n_qblocks * p.n_ftiles;
+  if (n_units > kMaxI32) return PBA_ERR_INVALID_ARG;
+  p.n_units = int(n_units);
+  p.masked = (key_mask != nullptr) || (N % pba::kBN != 0);
+  p.mask_vec4 = key_mask != nullptr && (reinterpret_cast<uintptr_t>(key_mask) & 3u) == 0;
+  p.mask = key_mask;
+  p.out = static_cast<uint16_t *>(out);
+  p.gate = static_cast<const uint16_t *>(gate);
+  p.lse = lse;
+  p.err = device_error_word();
+  if (p.err == nullptr) return PBA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return PBA_ERR_CUDA;
+  const int grid = int(std::min<int64_t>(n_units, sms));
+  cudaStream_t st = static_cast<cudaStream_t>(stream_ptr);
+  cudaError_t e = (D == 64) ? dispatch_pwa<64>(p, grid, gate != nullptr, st)
+                            : dispatch_pwa<32>(p, grid, gate != nullptr, st);
   return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
 }
 

@@ -28,7 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pba_status_string",
+    for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pwa_forward",
+              "pba_status_string",
               "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout",
               "pba_selftest_exp2"):
         assert n in names
@@ -41,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
         assert n in exported, n
         assert hasattr(lib, n)
     # nothing else of ours leaks out of the hidden-visibility build
-    ours = {s for s in exported if s.startswith(("pba", "softmax", "tri_"))}
+    ours = {s for s in exported if s.startswith(("pba", "softmax", "tri_", "pwa"))}
     assert ours == set(declared_functions())
 
 
@@ -161,6 +162,23 @@ def test_proj_rejects_null_and_unaligned(lib):
     bad = list(args)
     bad[0] = ctypes.c_void_p(0x10008)  # z not 16-byte aligned
     assert lib.tri_proj_forward(16, 128, 4, 32, *bad, None) == pba.PBA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("S,N,H,D,expect", [
+    (4, 64, 2, 16, pba.PBA_ERR_UNSUPPORTED),   # head dim
+    (4, 60, 2, 32, pba.PBA_ERR_INVALID_ARG),   # N not a multiple of 8
+    (-1, 64, 2, 32, pba.PBA_ERR_INVALID_ARG),
+    (4, 64, 0, 32, pba.PBA_ERR_INVALID_ARG),
+])
+def test_pwa_rejects_bad_shapes(lib, S, N, H, D, expect):
+    assert lib.pwa_forward(S, N, H, D, FAKE, FAKE, None, None, FAKE, None, None) == expect
+
+
+def test_pwa_rejects_null_and_unaligned(lib):
+    assert lib.pwa_forward(4, 64, 2, 32, None, FAKE, None, None, FAKE, None, None) == pba.PBA_ERR_INVALID_ARG
+    assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, None, None, None, None) == pba.PBA_ERR_INVALID_ARG
+    odd = ctypes.c_void_p(0x10008)
+    assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, odd, FAKE, None, None) == pba.PBA_ERR_INVALID_ARG
 
 
 def test_selftest_rejects_bad_limit(lib):
