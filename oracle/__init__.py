@@ -65,6 +65,8 @@ def _lib(mutant: int = 0):
             lib.oracle_tri_proj.restype = ctypes.c_int
             lib.oracle_pwa.argtypes = [_i64] * 4 + [_p] * 6 + [ctypes.c_int]
             lib.oracle_pwa.restype = ctypes.c_int
+            lib.oracle_pba_backward.argtypes = [_i64] * 5 + [_dbl] + [_p] * 10 + [ctypes.c_int]
+            lib.oracle_pba_backward.restype = ctypes.c_int
             lib.oracle_threads_used.argtypes = [ctypes.c_int]
             lib.oracle_threads_used.restype = ctypes.c_int
             _LIBS[mutant] = lib
@@ -238,3 +240,21 @@ def pwa(v, bias, key_mask=None, g=None, nthreads: int = 0, mutant: int = 0):
     rc = _lib(mutant).oracle_pwa(S, N, H, D, _ptr(vf), _ptr(bf), _ptr(gf), _ptr(mk), _ptr(out), _ptr(lse), nthreads)
     assert rc == 0
     return {"o": out, "lse": lse}
+
+
+def pba_backward(q, k, v, bias, dout, key_mask=None, softmax_scale=None, nthreads: int = 0, mutant: int = 0):
+    """Gradients of pair-biased attention in fp64 (see pba_oracle.c): q, dout
+    [B,H,Nq,D], k, v [B,H,Nk,D], bias [B,H,Nq,Nk] (broadcast views are
+    expanded), key_mask [B,Nk] or None.  Returns dq, dk, dv, dbias."""
+    qf, kf, vf, of = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, Nq, D = qf.shape
+    Nk = kf.shape[2]
+    bf = np.ascontiguousarray(np.broadcast_to(_f64(bias), (B, H, Nq, Nk)))
+    mk = _u8(key_mask)
+    dq, dk, dv = np.zeros_like(qf), np.zeros_like(kf), np.zeros_like(vf)
+    dbias = np.zeros((B, H, Nq, Nk))
+    rc = _lib(mutant).oracle_pba_backward(B, H, Nq, Nk, D, _default_tau(D, softmax_scale), _ptr(qf), _ptr(kf),
+                                          _ptr(vf), _ptr(bf), _ptr(mk), _ptr(of), _ptr(dq), _ptr(dk), _ptr(dv),
+                                          _ptr(dbias), nthreads)
+    assert rc == 0
+    return {"dq": dq, "dk": dk, "dv": dv, "dbias": dbias}

@@ -478,3 +478,93 @@ int oracle_pwa(int64_t S, int64_t N, int64_t H, int64_t D, const double *v, cons
   parallel_rows(pwa_row, &x, H * N, N, nthreads);
   return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Backward of pair-biased attention (training is distributed too:     */
+/* Fold-CP, Figure 3 right, training scaling).  For one (b, h), with    */
+/* s_ij = tau q_i.k_j + b_ij over valid keys and P_ij = exp(s_ij - lse_i)*/
+/* (0 for invalid keys), given dO = dL/dO:                              */
+/*   O_i      = sum_j P_ij v_j                                          */
+/*   Delta_i  = sum_d dO_id O_id                                        */
+/*   dP_ij    = dO_i . v_j                                              */
+/*   dS_ij    = P_ij (dP_ij - Delta_i)        = dL/ds_ij = dL/db_ij     */
+/*   dq_i     = tau sum_j dS_ij k_j,  dk_j = tau sum_i dS_ij q_i        */
+/*   dv_j     = sum_i P_ij dO_i                                         */
+/* Contiguous fp64: q, dO [B][H][Nq][D]; k, v [B][H][Nk][D]; bias and    */
+/* dbias [B][H][Nq][Nk]; key_mask [B][Nk] or NULL.  One (b, h) per call  */
+/* of the row function; dbias of invalid keys is 0.                     */
+/* ------------------------------------------------------------------ */
+typedef struct {
+  int64_t B, H, Nq, Nk, D;
+  double tau;
+  const double *q, *k, *v, *bias, *dout;
+  const uint8_t *mask;
+  double *dq, *dk, *dv, *dbias;
+} bwd_ctx;
+
+static void bwd_bh(const void *vctx, int64_t bh, double *scratch) {
+  const bwd_ctx *c = (const bwd_ctx *)vctx;
+  const int64_t Nq = c->Nq, Nk = c->Nk, D = c->D, b = bh / c->H;
+  const double *q = c->q + bh * Nq * D, *k = c->k + bh * Nk * D, *v = c->v + bh * Nk * D;
+  const double *bias = c->bias + bh * Nq * Nk, *dout = c->dout + bh * Nq * D;
+  const uint8_t *mask = c->mask ? c->mask + b * Nk : NULL;
+  double *dq = c->dq + bh * Nq * D, *dk = c->dk + bh * Nk * D, *dv = c->dv + bh * Nk * D;
+  double *dbias = c->dbias + bh * Nq * Nk;
+  double *p = scratch, *o = scratch + Nk;
+  for (int64_t x = 0; x < Nk * D; ++x) dk[x] = dv[x] = 0.0;
+  for (int64_t i = 0; i < Nq; ++i) {
+    double m = -INFINITY;
+    for (int64_t j = 0; j < Nk; ++j) {
+      const int valid = (mask == NULL || mask[j] != 0) && bias[i * Nk + j] != -INFINITY;
+      double s = -INFINITY;
+      if (valid) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += q[i * D + d] * k[j * D + d];
+        s = c->tau * dot + bias[i * Nk + j];
+      }
+      p[j] = s;
+      if (s > m) m = s;
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < Nk; ++j) {
+      p[j] = (p[j] == -INFINITY) ? 0.0 : exp(p[j] - m);
+      l += p[j];
+    }
+    for (int64_t j = 0; j < Nk; ++j) p[j] = (l > 0.0) ? p[j] / l : 0.0;
+    for (int64_t d = 0; d < D; ++d) {
+      o[d] = 0.0;
+      for (int64_t j = 0; j < Nk; ++j) o[d] += p[j] * v[j * D + d];
+    }
+    double delta = 0.0;
+    for (int64_t d = 0; d < D; ++d) delta += dout[i * D + d] * o[d];
+    for (int64_t d = 0; d < D; ++d) dq[i * D + d] = 0.0;
+    for (int64_t j = 0; j < Nk; ++j) {
+      double dp = 0.0;
+      for (int64_t d = 0; d < D; ++d) dp += dout[i * D + d] * v[j * D + d];
+#if ORACLE_MUTANT == 14 /* planted: the row term Delta dropped */
+      const double ds = p[j] * dp;
+#else
+      const double ds = p[j] * (dp - delta);
+#endif
+      dbias[i * Nk + j] = ds;
+      for (int64_t d = 0; d < D; ++d) {
+        dq[i * D + d] += c->tau * ds * k[j * D + d];
+#if ORACLE_MUTANT == 15 /* planted: dk without the scale */
+        dk[j * D + d] += ds * q[i * D + d];
+#else
+        dk[j * D + d] += c->tau * ds * q[i * D + d];
+#endif
+        dv[j * D + d] += p[j] * dout[i * D + d];
+      }
+    }
+  }
+}
+
+int oracle_pba_backward(int64_t B, int64_t H, int64_t Nq, int64_t Nk, int64_t D, double tau, const double *q,
+                        const double *k, const double *v, const double *bias, const uint8_t *key_mask,
+                        const double *dout, double *dq, double *dk, double *dv, double *dbias, int nthreads) {
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 0 || D < 1) return 1;
+  bwd_ctx c = {B, H, Nq, Nk, D, tau, q, k, v, bias, dout, key_mask, dq, dk, dv, dbias};
+  parallel_rows(bwd_bh, &c, B * H, Nk + D, nthreads);
+  return 0;
+}

@@ -455,6 +455,61 @@ def test_pwa_closed_forms():
     assert np.all(r["o"] == 0) and np.all(r["lse"] == -np.inf)
 
 
+# ---------------------------------------------------------------- backward
+# Gradients of the same definition (training: Fold-CP, Figure 3 right).
+# Pinned against torch autograd through its fp64 math-path attention (an
+# independent implementation) and against central finite differences of the
+# oracle's own forward on a tiny problem.
+def _autograd_reference(q, k, v, bias, mask, dout):
+    q, k, v, bias = (x.clone().requires_grad_(True) for x in (q, k, v, bias))
+    add = bias
+    if mask is not None:
+        add = bias + torch.where(mask.bool(), 0.0, -math.inf).to(torch.float64)[:, None, None, :]
+    with torch.nn.attention.sdpa_kernel(torch.nn.attention.SDPBackend.MATH):
+        o = F.scaled_dot_product_attention(q, k, v, attn_mask=add)
+    o.backward(dout)
+    return q.grad, k.grad, v.grad, bias.grad
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_backward_matches_torch_autograd(seed):
+    q, k, v, bias, mask = _rand_problem(B=2, H=2, Nq=19, Nk=29, D=8, seed=seed, mask_frac=0.25)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(seed + 9), dtype=torch.float64)
+    r = oracle.pba_backward(q, k, v, bias, dout, mask)
+    dq, dk, dv, db = _autograd_reference(q, k, v, bias, mask, dout)
+    for name, a, b in (("dq", r["dq"], dq), ("dk", r["dk"], dk), ("dv", r["dv"], dv), ("dbias", r["dbias"], db)):
+        assert np.abs(a - b.numpy()).max() < 1e-12, name
+
+
+def test_backward_finite_differences():
+    q, k, v, bias, mask = _rand_problem(B=1, H=1, Nq=3, Nk=5, D=2, seed=4, mask_frac=0.0)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(5), dtype=torch.float64)
+    r = oracle.pba_backward(q, k, v, bias, dout)
+    loss = lambda qq, kk, vv, bb: float((oracle.pba(qq, kk, vv, bb)["o"] * dout.numpy()).sum())
+    eps = 1e-6
+    for name, t, pos in (("dq", q, 0), ("dk", k, 1), ("dv", v, 2), ("dbias", bias, 3)):
+        flat = t.reshape(-1)
+        for idx in range(0, flat.numel(), max(1, flat.numel() // 5)):
+            args = [q, k, v, bias]
+            plus, minus = [a.clone() for a in args], [a.clone() for a in args]
+            plus[pos].reshape(-1)[idx] += eps
+            minus[pos].reshape(-1)[idx] -= eps
+            fd = (loss(*plus) - loss(*minus)) / (2 * eps)
+            assert abs(fd - r[name].reshape(-1)[idx]) < 1e-7, (name, idx)
+
+
+def test_backward_masked_keys_get_no_gradient():
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=7, Nk=13, D=4, seed=6, mask_frac=0.4)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7), dtype=torch.float64)
+    r = oracle.pba_backward(q, k, v, bias, dout, mask)
+    dead = (mask[0] == 0).numpy()
+    assert np.all(r["dbias"][..., dead] == 0) and np.all(r["dk"][:, :, dead] == 0) and np.all(r["dv"][:, :, dead] == 0)
+    # dbias rows sum to zero (softmax Jacobian), dq is tau * dbias @ k
+    assert np.abs(r["dbias"].sum(-1)).max() < 1e-12
+    tau = 1.0 / math.sqrt(4)
+    assert np.abs(r["dq"] - tau * np.einsum("bhij,bhjd->bhid", r["dbias"], k.numpy())).max() < 1e-12
+
+
 # ---------------------------------------------------------------- planted mistakes
 def _pin_suite(mutant):
     """Run a compact set of the pins against an oracle build; return the
@@ -506,6 +561,12 @@ def _pin_suite(mutant):
     o = torch.einsum("hij,sjhd->sihd", torch.softmax(logits, dim=-1), v)
     if np.abs(pw["o"] - o.numpy()).max() > 1e-12:
         fails += 1
+    q, k, v, bias, mask = _rand_problem(B=1, H=2, Nq=9, Nk=12, D=4, seed=8, mask_frac=0.2)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(3), dtype=torch.float64)
+    bw = oracle.pba_backward(q, k, v, bias, dout, mask, mutant=mutant)
+    ref = _autograd_reference(q, k, v, bias, mask, dout)
+    if any(np.abs(bw[n] - t.numpy()).max() > 1e-12 for n, t in zip(("dq", "dk", "dv", "dbias"), ref)):
+        fails += 1
     return fails
 
 
@@ -513,6 +574,6 @@ def test_default_build_passes_compact_pins():
     assert _pin_suite(0) == 0
 
 
-@pytest.mark.parametrize("mutant", range(1, 14))
+@pytest.mark.parametrize("mutant", range(1, 16))
 def test_planted_mistake_is_caught(mutant):
     assert _pin_suite(mutant) > 0, f"planted mistake {mutant} went unnoticed"
