@@ -214,6 +214,31 @@ PBA_API pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, 
 PBA_API pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v, const void *bias,
                                const uint8_t *key_mask, const void *gate, void *out, float *lse, void *stream);
 
+/*
+ * pba_backward -- gradients of pba_forward (training is distributed too:
+ * Fold-CP, Figure 3 right).  With s_ij = tau q_i.k_j + b_ij over valid keys,
+ * P_ij = exp(s_ij - lse_i) recomputed from the forward's log-sum-exp, and
+ * dout = dL/dO:
+ *   delta_i = sum_d dout_id out_id          (written: delta [B][H][Nq] float)
+ *   dS_ij   = P_ij (dout_i . v_j - delta_i) (written: dbias [B][H][Nq][Nk] bf16;
+ *                                            0 for masked keys and -inf bias)
+ *   dq_i = tau sum_j dS_ij k_j,  dk_j = tau sum_i dS_ij q_i,  dv_j = sum_i P_ij dout_i
+ *                                           (written: dq, dk, dv float, contiguous
+ *                                            [B][H][Nq or Nk][D])
+ * `desc` describes q, k, v, bias, key_mask, out, lse as for pba_forward; the
+ * output strides also describe dout.  bf16 only.  q, k, v, out, dout and the
+ * outputs must be contiguous [B][H][n][D], lse contiguous [B][H][Nq], the
+ * bias row stride and Nk multiples of 8, every pointer 16-byte aligned
+ * (else PBA_ERR_INVALID_ARG).  Nq = 0 or Nk = 0 writes nothing.  The caller
+ * owns every buffer, delta included; nothing is allocated.  Asynchronous on
+ * `stream`: one delta kernel, then one kernel for dq and dbias and one for dk
+ * and dv.
+ */
+PBA_API pba_status pba_backward(const pba_attn_desc *desc, const void *q, const void *k, const void *v,
+                                const void *bias, const uint8_t *key_mask, const void *out, const float *lse,
+                                const void *dout, float *dq, float *dk, float *dv, void *dbias, float *delta,
+                                void *stream);
+
 /* Human-readable name of a status code (static storage). */
 PBA_API const char *pba_status_string(pba_status status);
 

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "PbaError", "PBA_OK", "PBA_ERR_INVALID_ARG", "PBA_ERR_UNSUPPORTED", "PBA_ERR_CUDA", "PBA_ERR_TIMEOUT",
-    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pwa_forward",
+    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pwa_forward", "pba_backward",
     "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_selftest_exp2",
     "pba_status_string",
 ]
@@ -85,6 +85,8 @@ def load_library() -> ctypes.CDLL:
     lib.tri_proj_forward.restype = st
     lib.pwa_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 7
     lib.pwa_forward.restype = st
+    lib.pba_backward.argtypes = [desc_p] + [_p] * 14
+    lib.pba_backward.restype = st
     lib.pba_status_string.argtypes = [st]
     lib.pba_status_string.restype = ctypes.c_char_p
     lib.pba_last_device_error.argtypes = [_p]
@@ -332,6 +334,33 @@ def pwa_forward(v, bias, key_mask=None, gate=None, out=None, lse=None, return_ls
     _check("pwa_forward", load_library().pwa_forward(S, N, H, D, _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
                                                      _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def pba_backward(q, k, v, bias, key_mask, out, lse, dout, softmax_scale=None, stream=None):
+    """Gradients of pba_forward, bf16 inputs (contiguous [B,H,n,D]; bias as
+    for pba_forward).  Returns dq, dk, dv (fp32), dbias [B,H,Nq,Nk] (bf16) and
+    delta = rowsum(dout * out) [B,H,Nq] (fp32)."""
+    for n, t in (("out", out), ("dout", dout)):
+        _cuda(n, t, torch.bfloat16)
+    _cuda("lse", lse, torch.float32)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if out.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("out and dout must be [B,H,Nq,D], lse [B,H,Nq]")
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    dbias = torch.empty((B, H, Nq, Nk), dtype=torch.bfloat16, device=q.device)
+    delta = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    d = _desc(q, k, v, bias, key_mask, out.stride()[:3] if out.dim() == 4 else None, lse.stride(), softmax_scale)
+    _check("pba_backward", load_library().pba_backward(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(bias),
+                                                       _ptr(key_mask), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                                       _ptr(dk), _ptr(dv), _ptr(dbias), _ptr(delta),
+                                                       _stream(stream)))
+    return dq, dk, dv, dbias, delta
 
 
 def pba_last_device_error(stream=None) -> int:

@@ -16,6 +16,7 @@
 #include "pba_attn_sm100.cuh"
 #include "pba_proj_sm100.cuh"
 #include "pba_pwa_sm100.cuh"
+#include "pba_bwd_sm100.cuh"
 #include "pba_simt.cuh"
 
 // Device error word: written by kernels whose bounded waits ran out, read and
@@ -409,6 +410,26 @@ cudaError_t dispatch_pwa(const pba::PwaParams &p, int grid, bool gate, cudaStrea
   return m ? launch_pwa<D, false, true>(p, grid, st) : launch_pwa<D, false, false>(p, grid, st);
 }
 
+// ------------------------------------------------------------ backward
+template <int D, bool kB>
+cudaError_t launch_bwd(const pba::BwdParams &p, int grid, cudaStream_t stream) {
+  using L = pba::BwdLayout<D>;
+  auto kern = pba::pba_bwd_sm100_kernel<D, kB>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, pba::kBwdThreads, L::kSmemAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
+// Dense [B][H][N][D]; the stride of an extent-1 dimension does not matter.
+bool contiguous_bhnd(const int64_t s[3], int64_t B, int64_t H, int64_t N, int64_t D) {
+  return (N <= 1 || s[2] == D) && (H <= 1 || s[1] == N * D) && (B <= 1 || s[0] == H * N * D);
+}
+
 }  // namespace
 
 extern "C" {
@@ -626,6 +647,96 @@ pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v
   cudaError_t e = (D == 64) ? dispatch_pwa<64>(p, grid, gate != nullptr, st)
                             : dispatch_pwa<32>(p, grid, gate != nullptr, st);
   return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+pba_status pba_backward(const pba_attn_desc *d, const void *q, const void *k, const void *v, const void *bias,
+                        const uint8_t *key_mask, const void *out, const float *lse, const void *dout, float *dq,
+                        float *dk, float *dv, void *dbias, float *delta, void *stream_ptr) {
+  pba_status s = check_desc(d);
+  if (s != PBA_OK) return s;
+  if (d->dtype != PBA_BF16) return PBA_ERR_UNSUPPORTED;
+  const int64_t B = d->B, H = d->H, Nq = d->Nq, Nk = d->Nk, D = d->D;
+  if (Nq == 0 || Nk == 0) return PBA_OK;  // no scores: nothing to write (a caller zero-fills dk, dv or dq)
+  const void *ptrs[] = {q, k, v, bias, out, lse, dout, dq, dk, dv, dbias, delta};
+  for (const void *x : ptrs)
+    if (x == nullptr || !aligned16(x)) return PBA_ERR_INVALID_ARG;
+  // contiguous [B][H][n][D] tensors (the output strides describe out and dout)
+  if (!contiguous_bhnd(d->q_stride, B, H, Nq, D) || !contiguous_bhnd(d->k_stride, B, H, Nk, D) ||
+      !contiguous_bhnd(d->v_stride, B, H, Nk, D) || !contiguous_bhnd(d->out_stride, B, H, Nq, D))
+    return PBA_ERR_INVALID_ARG;
+  if ((Nq > 1 && d->lse_stride[2] != 1) || (H > 1 && d->lse_stride[1] != Nq) ||
+      (B > 1 && d->lse_stride[0] != H * Nq))
+    return PBA_ERR_INVALID_ARG;
+  if (d->bias_stride[2] % 8 != 0 || Nk % 8 != 0) return PBA_ERR_INVALID_ARG;  // 16-byte bias and dbias rows
+  if (B * H * Nq > kMaxI32 || B * H * Nk > kMaxI32) return PBA_ERR_INVALID_ARG;
+  s = check_device();
+  if (s != PBA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream_ptr);
+  pba::BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const CUtensorMapSwizzle swz = (D == 64) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const uint32_t box[4] = {uint32_t(D), uint32_t(pba::kBwdTile), 1, 1};
+  {
+    const uint64_t dq_[4] = {uint64_t(D), uint64_t(Nq), uint64_t(H), uint64_t(B)};
+    const uint64_t dk_[4] = {uint64_t(D), uint64_t(Nk), uint64_t(H), uint64_t(B)};
+    const int64_t sq[3] = {D * 2, Nq * D * 2, H * Nq * D * 2}, sk[3] = {D * 2, Nk * D * 2, H * Nk * D * 2};
+    if (!make_map(&p.tm_q, q, dq_, sq, box, swz) || !make_map(&p.tm_do, dout, dq_, sq, box, swz) ||
+        !make_map(&p.tm_k, k, dk_, sk, box, swz) || !make_map(&p.tm_v, v, dk_, sk, box, swz))
+      return PBA_ERR_INVALID_ARG;
+  }
+  const bool bh_bcast = d->bias_stride[1] == 0 && H > 1, bb_bcast = d->bias_stride[0] == 0 && B > 1;
+  const uint64_t bdims[4] = {uint64_t(Nk), uint64_t(Nq), bh_bcast ? 1 : uint64_t(H), bb_bcast ? 1 : uint64_t(B)};
+  const int64_t bst[3] = {d->bias_stride[2] * 2, d->bias_stride[1] * 2, d->bias_stride[0] * 2};
+  p.bias_h_bcast = bh_bcast;
+  p.bias_b_bcast = bb_bcast;
+  p.B = int(B);
+  p.H = int(H);
+  p.Nq = int(Nq);
+  p.Nk = int(Nk);
+  p.tau = tau_of(d->softmax_scale, D);
+  p.mask = key_mask;
+  p.mask_sb = d->mask_stride_b;
+  p.lse = lse;
+  p.delta = delta;
+  p.row_sb = H * Nq;
+  p.row_sh = Nq;
+  p.dbias = static_cast<uint16_t *>(dbias);
+  p.db_sb = H * Nq * Nk;
+  p.db_sh = Nq * Nk;
+  p.db_sn = Nk;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.err = device_error_word();
+  if (p.err == nullptr) return PBA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
+  // Delta = rowsum(dO * O)
+  const int64_t rows = B * H * Nq;
+  pba::pba_bwd_delta_kernel<<<int((rows * 32 + 255) / 256), 256, 0, st>>>(
+      static_cast<const uint16_t *>(dout), static_cast<const uint16_t *>(out), delta, rows, int(D));
+  if (cudaGetLastError() != cudaSuccess) return PBA_ERR_CUDA;
+  cudaError_t e;
+  {
+    // kernel A: dq and dbias, one CTA per (b, h, 128 query rows)
+    pba::BwdParams a = p;
+    const uint32_t bbox[4] = {64, uint32_t(pba::kBwdTile), 1, 1};
+    if (!make_map(&a.tm_bias, bias, bdims, bst, bbox, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+    a.n_tiles = int((Nq + pba::kBwdTile - 1) / pba::kBwdTile);
+    const int grid = int(B * H * a.n_tiles);
+    e = (D == 64) ? launch_bwd<64, false>(a, grid, st) : launch_bwd<32, false>(a, grid, st);
+    if (e != cudaSuccess) return PBA_ERR_CUDA;
+  }
+  {
+    // kernel B: dk and dv, one CTA per (b, h, 128 key rows)
+    pba::BwdParams bb = p;
+    const uint32_t bbox[4] = {uint32_t(pba::kBwdTile), uint32_t(pba::kBwdTile), 1, 1};
+    if (!make_map(&bb.tm_bias, bias, bdims, bst, bbox, CU_TENSOR_MAP_SWIZZLE_NONE)) return PBA_ERR_INVALID_ARG;
+    bb.n_tiles = int((Nk + pba::kBwdTile - 1) / pba::kBwdTile);
+    const int grid = int(B * H * bb.n_tiles);
+    e = (D == 64) ? launch_bwd<64, true>(bb, grid, st) : launch_bwd<32, true>(bb, grid, st);
+    if (e != cudaSuccess) return PBA_ERR_CUDA;
+  }
+  return PBA_OK;
 }
 
 const char *pba_status_string(pba_status status) {

@@ -1,0 +1,428 @@
+// pba_bwd_sm100.cuh -- backward of pair-biased attention on sm_100a.
+//
+// Training is distributed too ("Fold-CP: A Context Parallelism Framework for
+// Biomolecular Modeling", Figure 3 right, training scaling).  For one (b, h),
+// with s_ij = tau q_i.k_j + b_ij over valid keys, lse_i from the forward pass
+// and P_ij = exp(s_ij - lse_i) (0 for masked keys):
+//     Delta_i = sum_d dO_id O_id                        (pba_bwd_delta_kernel)
+//     dP_ij   = dO_i . v_j
+//     dS_ij   = P_ij (dP_ij - Delta_i) = dL/db_ij       (dbias, bf16)
+//     dq_i    = tau sum_j dS_ij k_j                      (kernel A, fp32)
+//     dk_j    = tau sum_i dS_ij q_i,  dv_j = sum_i P_ij dO_i   (kernel B, fp32)
+//
+// Kernel A walks the key tiles of one 128-row query tile: S = Q K^T and
+// dP = dO V^T on the tensor cores (fp32 in Tensor Memory), P and dS on the
+// CUDA cores, dS to HBM as dbias and to Tensor Memory as bf16, then
+// dQ += dS K (A = dS from Tensor Memory, B = the K tile read MN-major).
+// Kernel B walks the query tiles of one 128-row key tile: S^T = K Q^T and
+// dP^T = V dO^T, then dV += P^T dO and dK += dS^T Q with P^T and dS^T from
+// Tensor Memory and dO, Q read MN-major.  Both recompute P from the saved
+// log-sum-exp, so no N^2 intermediate is stored besides dbias.
+//
+// One CTA per unit, 192 threads: warps 0-3 the compute warpgroup (row =
+// thread = Tensor Memory lane), warp 4 the TMA producer, warp 5 Tensor Memory
+// and the MMAs.  The per-tile chain is sequential (S, dP -> P, dS -> dQ or
+// dV, dK); operand tiles are double-buffered.
+#pragma once
+
+#include <cuda.h>
+#include <cstdint>
+
+#include "pba_ptx.cuh"
+
+namespace pba {
+
+constexpr int kBwdThreads = 192;
+constexpr int kBwdTile = 128;
+
+struct BwdParams {
+  // A: tm_q/tm_do are the query-side tiles, tm_k/tm_v the key-side tiles;
+  // all 4-D (D, n, H, B) bf16 with box {D, 128, 1, 1}.  tm_bias: (Nk, Nq, H, B)
+  // bf16, kernel A box {64, 128} 128-byte swizzle, kernel B box {128, 128}
+  // no swizzle.
+  CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_bias;
+  int32_t B, H, Nq, Nk;
+  int32_t n_tiles;      // A: ceil(Nq/128), B: ceil(Nk/128) per (b, h)
+  int32_t bias_h_bcast, bias_b_bcast;  // bias head / batch stride 0 (map extent 1)
+  float tau;
+  const uint8_t *mask;  // [B][Nk] or null
+  int64_t mask_sb;
+  const float *lse, *delta;  // [B][H][Nq]
+  int64_t row_sb, row_sh;    // strides of lse / delta (elements); row stride 1
+  uint16_t *dbias;           // [B][H][Nq][Nk] bf16 (contiguous rows of Nk)
+  int64_t db_sb, db_sh, db_sn;
+  float *dq, *dk, *dv;       // fp32 [B][H][n][D] contiguous
+  int *err;
+  uint64_t timeout_ns;
+};
+
+template <int D>
+struct BwdLayout {
+  static_assert(D == 32 || D == 64, "head dimension");
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kSwizzleMode = (D == 64) ? 2 : 4;
+  static constexpr int kAtomBytes = 8 * kRowBytes;
+  static constexpr int kTileBytes = kBwdTile * kRowBytes;  // one [128][D] bf16 tile
+  static constexpr int kBiasBytes = kBwdTile * kBwdTile * 2;
+  static constexpr int kStages = 2;
+  // fixed operands of the unit (A: Q, dO; B: K, V), then per-step operands
+  // (A: K, V; B: Q, dO) and the bias tile, double-buffered
+  static constexpr int kOffFix0 = 0;
+  static constexpr int kOffFix1 = kOffFix0 + kTileBytes;
+  static constexpr int kOffStep0 = kOffFix1 + kTileBytes;                   // [stage]
+  static constexpr int kOffStep1 = kOffStep0 + kStages * kTileBytes;        // [stage]
+  static constexpr int kOffBias = kOffStep1 + kStages * kTileBytes;         // [stage]
+  // kernel B: log2-scaled lse and Delta of the step's 128 query columns,
+  // double-buffered by step parity
+  static constexpr int kOffRowv = kOffBias + kStages * kBiasBytes;
+  static constexpr int kOffBar = kOffRowv + 2 * 2 * kBwdTile * 4;
+  static constexpr int kBarFixFull = 0;
+  static constexpr int kBarStepFull = 1;                       // [stage]
+  static constexpr int kBarStepEmpty = kBarStepFull + kStages;  // [stage]
+  static constexpr int kBarSFull = kBarStepEmpty + kStages;
+  static constexpr int kBarSFree = kBarSFull + 1;
+  static constexpr int kBarGFull = kBarSFree + 1;  // P / dS written to Tensor Memory
+  static constexpr int kBarGDone = kBarGFull + 1;  // the accumulating MMAs of a step are done
+  static constexpr int kBarDrain = kBarGDone + 1;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+  static constexpr int kOffAbort = kOffTmemSlot + 4;
+  static constexpr int kBytes = kOffAbort + 4;
+  static constexpr int kSmemAlloc = kBytes + 1024;
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  // Tensor Memory columns
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColG0 = 256, kColG1 = 320, kColAcc0 = 384,
+                            kColAcc1 = 384 + D;
+  static_assert(kColAcc1 + D <= 512, "Tensor Memory budget");
+};
+
+// kB = false: kernel A (dq, dbias); kB = true: kernel B (dk, dv).
+template <int D, bool kB>
+__global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __grid_constant__ BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmemSlot);
+  int *abort_flag = reinterpret_cast<int *>(smem + L::kOffAbort);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // unit: (b, h, tile of 128 rows); steps: the tiles of the other side
+  const int unit = blockIdx.x;
+  const int tile = unit % p.n_tiles;
+  const int bh = unit / p.n_tiles;
+  const int h = bh % p.H, b = bh / p.H;
+  const int row0 = tile * kBwdTile;
+  const int n_other = kB ? p.Nq : p.Nk;
+  const int nsteps = (n_other + kBwdTile - 1) / kBwdTile;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[L::kBarFixFull], 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(&bars[L::kBarStepFull + s], 1);
+      mbar_init(&bars[L::kBarStepEmpty + s], 2);  // the MMA commit + the compute warpgroup (bias, row values)
+    }
+    mbar_init(&bars[L::kBarSFull], 1);
+    mbar_init(&bars[L::kBarSFree], kBwdTile);
+    mbar_init(&bars[L::kBarGFull], kBwdTile);
+    mbar_init(&bars[L::kBarGDone], 1);
+    mbar_init(&bars[L::kBarDrain], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{abort_flag, p.err, p.timeout_ns};
+  WaitCtl wc_drain = wc;
+  int drain_abort = 0;
+  wc_drain.abort_flag = &drain_abort;
+
+  if (warp == 4) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      const uint64_t pol = l2_policy_evict_last();
+      // fixed tiles of the unit: A: Q, dO rows; B: K, V rows
+      mbar_arrive_expect_tx(&bars[L::kBarFixFull], 2 * L::kTileBytes);
+      tma_load_4d(smem + L::kOffFix0, kB ? &p.tm_k : &p.tm_q, &bars[L::kBarFixFull], 0, row0, h, b, pol);
+      tma_load_4d(smem + L::kOffFix1, kB ? &p.tm_v : &p.tm_do, &bars[L::kBarFixFull], 0, row0, h, b, pol);
+      bool ok = true;
+      int it = 0;
+      for (; it < nsteps && ok; ++it) {
+        const int s = it % L::kStages;
+        if (it >= L::kStages) ok = mbar_wait(&bars[L::kBarStepEmpty + s], ((it / L::kStages) - 1) & 1, wc);
+        if (!ok) break;
+        const int o0 = it * kBwdTile;
+        uint64_t *full = &bars[L::kBarStepFull + s];
+        mbar_arrive_expect_tx(full, 2 * L::kTileBytes + L::kBiasBytes);
+        tma_load_4d(smem + L::kOffStep0 + s * L::kTileBytes, kB ? &p.tm_q : &p.tm_k, full, 0, o0, h, b, pol);
+        tma_load_4d(smem + L::kOffStep1 + s * L::kTileBytes, kB ? &p.tm_do : &p.tm_v, full, 0, o0, h, b, pol);
+        uint8_t *bdst = smem + L::kOffBias + s * L::kBiasBytes;
+        const int hb = p.bias_h_bcast ? 0 : h, bb = p.bias_b_bcast ? 0 : b;
+        if (kB) {
+          // [128 queries][128 keys], no swizzle: the thread of key j reads column j
+          tma_load_4d(bdst, &p.tm_bias, full, row0, o0, hb, bb, pol);
+        } else {
+          // [128 queries][128 keys] as two 64-key boxes, 128-byte swizzle
+          tma_load_4d(bdst, &p.tm_bias, full, o0, row0, hb, bb, pol);
+          tma_load_4d(bdst + L::kBiasBytes / 2, &p.tm_bias, full, o0 + 64, row0, hb, bb, pol);
+        }
+      }
+      mbar_wait(&bars[L::kBarFixFull], 0, wc_drain);
+      if (!ok)
+        for (int s = 0; s < L::kStages; ++s) {
+          const int a = (it - s + L::kStages - 1) / L::kStages;
+          if (a > 0) mbar_wait(&bars[L::kBarStepFull + s], (a - 1) & 1, wc_drain);
+        }
+    }
+  } else if (warp == 5) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kBwdTile, kBwdTile, false);  // both operands K-major
+      const uint32_t idesc_g = idesc_bf16_f32(kBwdTile, D, true);          // B MN-major
+      constexpr uint32_t kHi = smem_desc_hi(L::kAtomBytes, L::kSwizzleMode);
+      const uint32_t sF0 = smem_u32(smem + L::kOffFix0), sF1 = smem_u32(smem + L::kOffFix1);
+      bool ok = mbar_wait(&bars[L::kBarFixFull], 0, wc);
+      for (int it = 0; it < nsteps && ok; ++it) {
+        const int s = it % L::kStages;
+        ok = mbar_wait(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
+        // S and dP of the previous step must have been read
+        if (ok && it > 0) ok = mbar_wait(&bars[L::kBarSFree], (it - 1) & 1, wc);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
+        const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
+        // A: S = Q K^T, dP = dO V^T;  B: S^T = K Q^T, dP^T = V dO^T
+        const uint32_t a0 = smem_desc_lo(sF0, 16), b0 = smem_desc_lo(sS0, 16);
+        const uint32_t a1 = smem_desc_lo(sF1, 16), b1 = smem_desc_lo(sS1, 16);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem + L::kColS, desc_join(a0 + kk * 2, kHi), desc_join(b0 + kk * 2, kHi), idesc_s, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_bf16_ss(tmem + L::kColDP, desc_join(a1 + kk * 2, kHi), desc_join(b1 + kk * 2, kHi), idesc_s, kk > 0);
+        tc_commit(&bars[L::kBarSFull]);
+        // the accumulating products once P / dS are in Tensor Memory
+        ok = mbar_wait(&bars[L::kBarGFull], it & 1, wc);
+        if (!ok) break;
+        tc_fence_after_sync();
+        const uint32_t acc = (it > 0) ? 1u : 0u;
+        if (!kB) {
+          // dQ += dS K: B = the K tile, keys are the reduction (MN-major read)
+          const uint32_t kb = smem_desc_lo(sS0, L::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBwdTile / 16; ++kk)
+            mma_bf16_ts(tmem + L::kColAcc0, tmem + L::kColG0 + kk * 8,
+                        desc_join(kb + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
+        } else {
+          // dV += P^T dO and dK += dS^T Q: queries are the reduction
+          const uint32_t qb = smem_desc_lo(sS0, L::kTileBytes), ob = smem_desc_lo(sS1, L::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBwdTile / 16; ++kk)
+            mma_bf16_ts(tmem + L::kColAcc1, tmem + L::kColG0 + kk * 8,
+                        desc_join(ob + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < kBwdTile / 16; ++kk)
+            mma_bf16_ts(tmem + L::kColAcc0, tmem + L::kColG1 + kk * 8,
+                        desc_join(qb + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars[L::kBarGDone]);
+        tc_commit(&bars[L::kBarStepEmpty + s]);
+      }
+      tc_commit(&bars[L::kBarDrain]);
+      mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
+    }
+  } else {
+    // ================================================================ compute warpgroup
+    const int t = threadIdx.x;  // row of the unit's tile = Tensor Memory lane
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const int r = row0 + t;     // A: query row; B: key row
+    const float l2e = 1.4426950408889634f;
+    const float c_s = p.tau * l2e;
+    const uint8_t *mrow = p.mask ? p.mask + int64_t(b) * p.mask_sb : nullptr;
+    // A: this row's lse and Delta; B: this key's mask flag
+    float lse2 = 0.f, delta = 0.f;
+    bool key_ok = true;
+    if (!kB) {
+      if (r < p.Nq) {
+        const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + r;
+        lse2 = p.lse[at] * l2e;
+        delta = p.delta[at];
+      }
+    } else {
+      key_ok = r < p.Nk && (mrow == nullptr || mrow[r] != 0);
+    }
+    bool ok = true;
+    for (int it = 0; it < nsteps && ok; ++it) {
+      const int s = it % L::kStages;
+      const int o0 = it * kBwdTile;
+      // S, dP and the step's tiles, and the previous step's accumulating MMAs
+      // (they read G0/G1, which this step overwrites).  The waits only set ok;
+      // the warpgroup leaves together at the barrier below.
+      ok = mbar_wait<false>(&bars[L::kBarSFull], it & 1, wc);
+      if (ok) ok = mbar_wait<false>(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
+      if (ok && it > 0) ok = mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc);
+      const uint8_t *bt = smem + L::kOffBias + s * L::kBiasBytes;
+      // Per-step column data.  A: a keep bit per key (bit c>>2 of word c&3,
+      // from one ballot per 4 keys).  B: lse and Delta of the query columns,
+      // staged in shared memory by the warpgroup; the barrier also makes the
+      // warps leave the loop together.
+      uint32_t keepw[4] = {~0u, ~0u, ~0u, ~0u};
+      const float *rv = reinterpret_cast<const float *>(smem + L::kOffRowv) + (it & 1) * 2 * kBwdTile;
+      if (!kB) {
+        const int k0 = o0 + 4 * lane;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          keepw[e] = __ballot_sync(0xffffffffu, k0 + e < p.Nk && (mrow == nullptr || mrow[k0 + e] != 0));
+      } else {
+        const int qi = o0 + t;
+        const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
+        float *wv = const_cast<float *>(rv);
+        wv[t] = qi < p.Nq ? p.lse[at] * l2e : INFINITY;  // +inf: column past Nq (P = 0)
+        wv[kBwdTile + t] = qi < p.Nq ? p.delta[at] : 0.f;
+      }
+      ok = named_bar_and(1, kBwdTile, ok);
+      if (!ok) break;
+      tc_fence_after_sync();
+      // two halves of 64 columns: S, dP -> P, dS
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t sv[64], dpv[64];
+        tmem_ld32(tmem + lane_base + L::kColS + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tmem + lane_base + L::kColS + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tmem + lane_base + L::kColDP + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
+        tmem_ld32(tmem + lane_base + L::kColDP + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
+        tmem_wait_ld();
+        uint32_t pk[32], dk[32];
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          // eight columns: bias values and the column terms
+          float bv[8], l2v[8], dlv[8];
+          bool valid[8];
+          if (!kB) {
+            // 128-byte swizzled [query][key] tile: keys 8 c8 .. of row t
+            const int c = hf * 64 + c8 * 8, box = c >> 6, chunk = (c & 63) >> 3;
+            const uint4 w4 = *reinterpret_cast<const uint4 *>(bt + box * (L::kBiasBytes / 2) + t * 128 +
+                                                              ((chunk ^ (t & 7)) << 4));
+            const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              bv[e] = (e & 1) ? bf16hi_to_f32(ww[e >> 1]) : bf16lo_to_f32(ww[e >> 1]);
+              const int cc = c + e;
+              valid[e] = ((keepw[cc & 3] >> (cc >> 2)) & 1u) && r < p.Nq;
+              l2v[e] = lse2;
+              dlv[e] = delta;
+            }
+          } else {
+            // plain [query][key] tile: queries 8 c8 .. of key column t
+            const int c = hf * 64 + c8 * 8;
+            const float4 la = *reinterpret_cast<const float4 *>(rv + c), lb = *reinterpret_cast<const float4 *>(rv + c + 4);
+            const float4 da = *reinterpret_cast<const float4 *>(rv + kBwdTile + c);
+            const float4 db = *reinterpret_cast<const float4 *>(rv + kBwdTile + c + 4);
+            const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+            const float dv8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              bv[e] = __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t *>(bt + (c + e) * 256 + t * 2)) << 16);
+              valid[e] = key_ok;  // columns past Nq carry lse = +inf, so P = 0 there
+              l2v[e] = lv[e];
+              dlv[e] = dv8[e];
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int ee = c8 * 8 + e;
+            float pe = 0.f, ds = 0.f;
+            if (valid[e] && bv[e] != -INFINITY) {
+              pe = ex2_approx(fmaf(__uint_as_float(sv[ee]), c_s, fmaf(bv[e], l2e, -l2v[e])));
+              ds = pe * (__uint_as_float(dpv[ee]) - dlv[e]);
+            }
+            if (e & 1) {
+              pk[ee >> 1] |= pack_bf16x2(0.f, pe) & 0xFFFF0000u;
+              dk[ee >> 1] |= pack_bf16x2(0.f, ds) & 0xFFFF0000u;
+            } else {
+              pk[ee >> 1] = pack_bf16x2(pe, 0.f) & 0xFFFFu;
+              dk[ee >> 1] = pack_bf16x2(ds, 0.f) & 0xFFFFu;
+            }
+          }
+        }
+        if (!kB) {
+          // dbias row segment (64 keys) and dS into Tensor Memory
+          const int key0 = o0 + hf * 64;
+          if (r < p.Nq) {
+            uint16_t *dst = p.dbias + int64_t(b) * p.db_sb + int64_t(h) * p.db_sh + int64_t(r) * p.db_sn + key0;
+            if (key0 + 64 <= p.Nk) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                reinterpret_cast<uint4 *>(dst)[q] = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+            } else {
+              for (int e = 0; key0 + e < p.Nk; ++e) dst[e] = uint16_t((e & 1) ? (dk[e >> 1] >> 16) : (dk[e >> 1] & 0xFFFFu));
+            }
+          }
+          tmem_st32(tmem + lane_base + L::kColG0 + hf * 32, dk);
+        } else {
+          tmem_st32(tmem + lane_base + L::kColG0 + hf * 32, pk);  // P^T
+          tmem_st32(tmem + lane_base + L::kColG1 + hf * 32, dk);  // dS^T
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&bars[L::kBarSFree]);
+      mbar_arrive(&bars[L::kBarGFull]);
+      if (t == 0) mbar_arrive(&bars[L::kBarStepEmpty + s]);  // bias tile read
+    }
+    // -------------------------------------------------------------- epilogue
+    if (ok) ok = mbar_wait<false>(&bars[L::kBarGDone], (nsteps - 1) & 1, wc);
+    ok = named_bar_and(1, kBwdTile, ok);  // every thread gets here; the loads below are warp-collective
+    if (ok) {
+      tc_fence_after_sync();
+      const int nrows = kB ? p.Nk : p.Nq;
+#pragma unroll 1
+      for (int a = 0; a < (kB ? 2 : 1); ++a) {
+        // A: dQ (acc0, scaled by tau).  B: a = 0 dK (acc0, scaled by tau), a = 1 dV (acc1)
+        const uint32_t col = (a == 0) ? L::kColAcc0 : L::kColAcc1;
+        const float scale = (a == 0) ? p.tau : 1.f;
+        float *dst = !kB ? p.dq : (a == 0 ? p.dk : p.dv);
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + col + c, v);
+          tmem_wait_ld();
+          if (r < nrows) {
+            float4 *o = reinterpret_cast<float4 *>(dst + ((int64_t(b) * p.H + h) * nrows + r) * D + c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              o[q] = make_float4(__uint_as_float(v[4 * q]) * scale, __uint_as_float(v[4 * q + 1]) * scale,
+                                 __uint_as_float(v[4 * q + 2]) * scale, __uint_as_float(v[4 * q + 3]) * scale);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+// Delta_i = sum_d dO_id O_id (bf16 inputs, fp32 sum), one warp per row.
+__global__ void pba_bwd_delta_kernel(const uint16_t *dout, const uint16_t *out, float *delta, int64_t rows, int D) {
+  const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int d = lane; d < D; d += 32)
+    acc += __uint_as_float(uint32_t(dout[row * D + d]) << 16) * __uint_as_float(uint32_t(out[row * D + d]) << 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) delta[row] = acc;
+}
+
+}  // namespace pba
