@@ -21,8 +21,10 @@
 //
 // One CTA per unit, 192 threads: warps 0-3 the compute warpgroup (row =
 // thread = Tensor Memory lane), warp 4 the TMA producer, warp 5 Tensor Memory
-// and the MMAs.  The per-tile chain is sequential (S, dP -> P, dS -> dQ or
-// dV, dK); operand tiles are double-buffered.
+// and the MMAs.  Per step the chain is S, dP -> P, dS -> dQ or dV, dK; the
+// next step's S, dP are issued as soon as this step's have been read, so they
+// overlap the second half of the elementwise work.  Operand tiles are
+// double-buffered.
 #pragma once
 
 #include <cuda.h>
@@ -188,17 +190,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       const uint32_t idesc_g = idesc_bf16_f32(kBwdTile, D, true);          // B MN-major
       constexpr uint32_t kHi = smem_desc_hi(L::kAtomBytes, L::kSwizzleMode);
       const uint32_t sF0 = smem_u32(smem + L::kOffFix0), sF1 = smem_u32(smem + L::kOffFix1);
-      bool ok = mbar_wait(&bars[L::kBarFixFull], 0, wc);
-      for (int it = 0; it < nsteps && ok; ++it) {
+      // S, dP of step `it` (A: S = Q K^T, dP = dO V^T; B: S^T = K Q^T,
+      // dP^T = V dO^T) once its tiles have landed and the compute warpgroup has
+      // read the previous step's S and dP
+      auto issue_s = [&](int it) -> bool {
         const int s = it % L::kStages;
-        ok = mbar_wait(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
-        // S and dP of the previous step must have been read
-        if (ok && it > 0) ok = mbar_wait(&bars[L::kBarSFree], (it - 1) & 1, wc);
-        if (!ok) break;
+        if (!mbar_wait(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc)) return false;
+        if (it > 0 && !mbar_wait(&bars[L::kBarSFree], (it - 1) & 1, wc)) return false;
         tc_fence_after_sync();
         const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
         const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
-        // A: S = Q K^T, dP = dO V^T;  B: S^T = K Q^T, dP^T = V dO^T
         const uint32_t a0 = smem_desc_lo(sF0, 16), b0 = smem_desc_lo(sS0, 16);
         const uint32_t a1 = smem_desc_lo(sF1, 16), b1 = smem_desc_lo(sS1, 16);
 #pragma unroll
@@ -208,10 +209,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
         for (int kk = 0; kk < D / 16; ++kk)
           mma_bf16_ss(tmem + L::kColDP, desc_join(a1 + kk * 2, kHi), desc_join(b1 + kk * 2, kHi), idesc_s, kk > 0);
         tc_commit(&bars[L::kBarSFull]);
+        return true;
+      };
+      // Software-pipelined: S, dP of step it+1 go out as soon as step it's
+      // S, dP have been read, before the accumulating products of step it.
+      bool ok = mbar_wait(&bars[L::kBarFixFull], 0, wc);
+      if (ok) ok = issue_s(0);
+      for (int it = 0; it < nsteps && ok; ++it) {
+        const int s = it % L::kStages;
+        if (it + 1 < nsteps && !(ok = issue_s(it + 1))) break;
         // the accumulating products once P / dS are in Tensor Memory
         ok = mbar_wait(&bars[L::kBarGFull], it & 1, wc);
         if (!ok) break;
         tc_fence_after_sync();
+        const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
+        const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
         const uint32_t acc = (it > 0) ? 1u : 0u;
         if (!kB) {
           // dQ += dS K: B = the K tile, keys are the reduction (MN-major read)
@@ -299,6 +311,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
         tmem_ld32(tmem + lane_base + L::kColDP + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
         tmem_ld32(tmem + lane_base + L::kColDP + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
         tmem_wait_ld();
+        if (hf == 1) {
+          // S and dP are in registers: the next step's S, dP may overwrite them
+          tc_fence_before_sync();
+          mbar_arrive(&bars[L::kBarSFree]);
+        }
         uint32_t pk[32], dk[32];
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
@@ -373,7 +390,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       }
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&bars[L::kBarSFree]);
       mbar_arrive(&bars[L::kBarGFull]);
       if (t == 0) mbar_arrive(&bars[L::kBarStepEmpty + s]);  // bias tile read
     }
