@@ -48,3 +48,70 @@ def test_job_throughput_counts_every_rank():
 
 def test_single_rank_needs_no_group():
     assert bench.max_over_ranks(4.2, False) == 4.2
+
+
+# ---------------------------------------------------------------- ring attention schedule (gloo, CPU)
+def _oracle_partial(q, k, v, bias, key_mask, softmax_scale=None, stream=None):
+    import oracle
+    r = oracle.pba_partial(q, k, v, bias, key_mask, softmax_scale)
+    return tuple(torch.from_numpy(r[n]) for n in ("o", "m", "l"))
+
+
+def _oracle_merge(o, m, l, out_dtype=None, stream=None):
+    import oracle
+    r = oracle.merge(o, m, l)
+    return torch.from_numpy(r["o"]), torch.from_numpy(r["lse"])
+
+
+def _ring_problem(P, B=1, H=2, L=24, D=8, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    N = P * L
+    q = torch.randn(B, H, N, D, generator=g, dtype=torch.float64)
+    k = torch.randn(B, H, N, D, generator=g, dtype=torch.float64)
+    v = torch.randn(B, H, N, D, generator=g, dtype=torch.float64)
+    bias = torch.randn(B, H, N, N, generator=g, dtype=torch.float64)
+    mask = (torch.rand(B, N, generator=g) > 0.2).to(torch.uint8)
+    return q, k, v, bias, mask
+
+
+def _ring_rank(rank, world, port, out):
+    from pair_biased_attention_b200 import ring
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        q, k, v, bias, mask = _ring_problem(world)
+        L = k.shape[2] // world
+        rows = slice(rank * L, (rank + 1) * L)
+        o, lse = ring.ring_attention(q[:, :, rows], k[:, :, rows], v[:, :, rows], bias[:, :, rows], mask,
+                                     partial_fn=_oracle_partial, merge_fn=_oracle_merge)
+        out[rank] = (o.numpy(), lse.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_attention_schedule_equals_full_attention(world):
+    """The distributed ring (point-to-point rotation of the key/value blocks,
+    one partial per step, tiled-softmax merge) gives each rank the attention
+    of its rows against all keys."""
+    import oracle
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_ring_rank, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
+    q, k, v, bias, mask = _ring_problem(world)
+    ref = oracle.pba(q, k, v, bias, mask)
+    L = k.shape[2] // world
+    for r in range(world):
+        o, lse = out[r]
+        assert abs(o - ref["o"][:, :, r * L:(r + 1) * L]).max() < 1e-12
+        assert abs(lse - ref["lse"][:, :, r * L:(r + 1) * L]).max() < 1e-12
+
+
+def test_ring_block_order():
+    from pair_biased_attention_b200 import ring
+    assert ring.ring_block_order(4, 0) == [0, 3, 2, 1]
+    assert ring.ring_block_order(4, 2) == [2, 1, 0, 3]
+    for P in (1, 2, 5):
+        for r in range(P):
+            assert sorted(ring.ring_block_order(P, r)) == list(range(P))
