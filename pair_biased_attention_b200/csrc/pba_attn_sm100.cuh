@@ -507,6 +507,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           for (int c8 = 0; c8 < kPre; ++c8)
             bpre[c8] = *reinterpret_cast<const uint4 *>(tile + t * 128 + ((c8 ^ (t & 7)) << 4));
         }
+        uint4 kpre[kMasked && !kBiasT ? kPre : 1];  // and their mask words
+        if (kMasked && !kBiasT) {
+#pragma unroll
+          for (int c8 = 0; c8 < kPre; ++c8)
+            kpre[c8] = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
+        }
 
         ok = mbar_wait<false>(&bars[L::kBarSFull + w], gt & 1, wc);
         if (!ok) break;
@@ -541,7 +547,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
             uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
             if (kMasked) {
               // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
-              const uint4 kv = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
+              const uint4 kv = c8 < kPre ? kpre[c8 < kPre ? c8 : 0]
+                                         : reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
               const uint32_t keep[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) wv[e] = (wv[e] & keep[e]) | (~keep[e] & 0xFF80FF80u);
