@@ -197,8 +197,8 @@ PBA_API pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, 
 /*
  * pwa_forward -- pair weighted averaging (Fold-CP, Table 1 row "Pair
  * Weighted Avg.", serial time B*H*S*N^2*D, distributed as a "2D ring + tiled
- * softmax"; Figure 2: it shares the softmax-merge archetype of the ring
- * attention).  The pages print no formula; the reading implemented here is a
+ * softmax"; Figure 2 groups it with the ring attention, a softmax whose
+ * per-block partials are merged).  The pages print no formula; the reading implemented here is a
  * softmax over the pair-bias logits alone, shared by the S sequences:
  *   w[h][i][:]    = softmax_j( bias[h][i][j] )  over keys j with key_mask[j] != 0
  *   o[s][i][h][:] = sum_j w[h][i][j] v[s][j][h][:]

@@ -419,8 +419,8 @@ int oracle_tri_proj(int64_t rows, int64_t c, int64_t F, int64_t H, const double 
 /* ------------------------------------------------------------------ */
 /* Pair weighted averaging (Fold-CP, Table 1 row "Pair Weighted Avg.": */
 /* serial time B*H*S*N^2*D, distributed as a "2D ring + tiled softmax", */
-/* and Figure 2: it shares the softmax-merge archetype of the ring      */
-/* attention).  The pages give no formula; the reading used here is a   */
+/* and Figure 2, which groups it with the ring attention: a softmax    */
+/* whose per-block partials are merged).  The pages give no formula; the reading used here is a   */
 /* softmax over the pair-bias logits alone, shared by the S sequences:  */
 /*   w[h][i][j] = exp(b[h][i][j] - m) / l  over valid keys j            */
 /*     (m = max, l = sum of exp(b - m) over valid j of row (h, i))      */

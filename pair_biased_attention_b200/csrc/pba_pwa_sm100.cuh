@@ -3,7 +3,8 @@
 // For S sequences of N tokens and H heads ("Fold-CP: A Context Parallelism
 // Framework for Biomolecular Modeling", Table 1 row "Pair Weighted Avg.",
 // serial time B*H*S*N^2*D, distributed as a "2D ring + tiled softmax", and
-// Figure 2: it shares the softmax-merge archetype of the ring attention):
+// Figure 2, which groups it with the ring attention as a softmax whose
+// partials are merged):
 //     w[h][i][:]    = softmax_j( b[h][i][j] + mask_j )      (bias [H][N][N])
 //     o[s][i][h][:] = sum_j w[h][i][j] v[s][j][h][:]        (v [S][N][H][D])
 //     out = o * sigmoid(g) (gate [S][N][H][D], optional); lse[h][i] (optional)

@@ -1,9 +1,10 @@
 """Context-parallel pair-biased attention over a 1D ring of ranks.
 
 "Fold-CP: A Context Parallelism Framework for Biomolecular Modeling",
-Figure 2(c) ("Ring Attention Pair Bias: 1D ring rotation of keys, values,
-and pair bias with tiled-softmax merge") and Table 1 (ring patterns take P
-steps, double-buffered).  Rank r of P holds the query rows of block r, the
+Figure 2(c): the keys, values and pair bias of the attention move around a
+one-dimensional ring of ranks and the per-step partials are combined by a
+tiled-softmax merge; Table 1's caption adds that each ring takes P steps with
+the next transfer overlapped.  Rank r of P holds the query rows of block r, the
 key/value rows of block r, and its own rows of the pair bias against every
 key (the row sharding of "Design-CP: Context Parallelism for Design of
 Protein Nanoparticles"), so only the key/value blocks travel around the ring.

@@ -398,7 +398,7 @@ def test_proj_linearity_and_row_selection():
 
 # ---------------------------------------------------------------- pair weighted averaging
 # Fold-CP, Table 1 row "Pair Weighted Avg." (B*H*S*N^2*D; "2D ring + tiled
-# softmax") and Figure 2 (shares the softmax-merge archetype).  Reading: a
+# softmax") and Figure 2 (grouped with the ring attention's merged softmax).  Reading: a
 # softmax over the pair-bias logits alone, shared by the S sequences.  Pinned
 # against pair-biased attention with zero queries (a different oracle path),
 # torch's fp64 softmax and einsum, and closed forms.
