@@ -3,7 +3,6 @@ runs the same workload, the job time is the maximum over ranks and the rate
 counts every rank's work.  The kernels are not involved: the path has no
 data-path collective (replicas of independent problems)."""
 import os
-import socket
 
 import pytest
 import torch
@@ -13,15 +12,13 @@ import torch.multiprocessing as mp
 import bench
 
 
-def _free_port():
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
+def _init(rank, world, rendezvous):
+    # a file rendezvous: no TCP port to collide with other processes
+    dist.init_process_group("gloo", init_method=f"file://{rendezvous}", rank=rank, world_size=world)
 
 
-def _rank_main(rank, world, port, times_ms, out):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+def _rank_main(rank, world, rendezvous, times_ms, out):
+    _init(rank, world, rendezvous)
     try:
         t = bench.max_over_ranks(times_ms[rank], True, device="cpu")
         out[rank] = t
@@ -31,11 +28,11 @@ def _rank_main(rank, world, port, times_ms, out):
 
 
 @pytest.mark.parametrize("world", [2])
-def test_job_time_is_max_over_ranks(world):
+def test_job_time_is_max_over_ranks(world, tmp_path):
     times = [3.0, 7.5][:world]
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_rank_main, args=(world, _free_port(), times, out), nprocs=world, join=True,
+    mp.start_processes(_rank_main, args=(world, str(tmp_path / "rdv"), times, out), nprocs=world, join=True,
                        start_method="spawn")
     assert [out[r] for r in range(world)] == [max(times)] * world
 
@@ -74,10 +71,9 @@ def _ring_problem(P, B=1, H=2, L=24, D=8, seed=0):
     return q, k, v, bias, mask
 
 
-def _ring_rank(rank, world, port, out):
+def _ring_rank(rank, world, rendezvous, out):
     from pair_biased_attention_b200 import ring
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    _init(rank, world, rendezvous)
     try:
         q, k, v, bias, mask = _ring_problem(world)
         L = k.shape[2] // world
@@ -91,14 +87,15 @@ def _ring_rank(rank, world, port, out):
 
 
 @pytest.mark.parametrize("world", [2, 3])
-def test_ring_attention_schedule_equals_full_attention(world):
+def test_ring_attention_schedule_equals_full_attention(world, tmp_path):
     """The distributed ring (point-to-point rotation of the key/value blocks,
     one partial per step, tiled-softmax merge) gives each rank the attention
     of its rows against all keys."""
     import oracle
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_ring_rank, args=(world, _free_port(), out), nprocs=world, join=True, start_method="spawn")
+    mp.start_processes(_ring_rank, args=(world, str(tmp_path / "rdv"), out), nprocs=world, join=True,
+                       start_method="spawn")
     q, k, v, bias, mask = _ring_problem(world)
     ref = oracle.pba(q, k, v, bias, mask)
     L = k.shape[2] // world
