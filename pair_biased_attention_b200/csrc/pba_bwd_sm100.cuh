@@ -264,7 +264,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     if (!kB) {
       if (r < p.Nq) {
         const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + r;
-        lse2 = p.lse[at] * l2e;
+        // a row with no valid key (lse = -inf) has -inf exponents for every
+        // key already; a finite stand-in keeps -lse from forming inf - inf
+        const float lse = p.lse[at];
+        lse2 = (lse == -INFINITY) ? 0.f : lse * l2e;
         delta = p.delta[at];
       }
     } else {
@@ -281,28 +284,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       if (ok) ok = mbar_wait<false>(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
       if (ok && it > 0) ok = mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc);
       const uint8_t *bt = smem + L::kOffBias + s * L::kBiasBytes;
-      // Per-step column data.  A: a keep bit per key (bit c>>2 of word c&3,
-      // from one ballot per 4 keys).  B: lse and Delta of the query columns,
-      // staged in shared memory by the warpgroup; the barrier also makes the
-      // warps leave the loop together.
-      uint32_t keepw[4] = {~0u, ~0u, ~0u, ~0u};
-      const float *rv = reinterpret_cast<const float *>(smem + L::kOffRowv) + (it & 1) * 2 * kBwdTile;
+      // Per-step column data in shared memory (double-buffered by step
+      // parity), written by the warpgroup; the barrier also makes the warps
+      // leave the loop together.  A: one keep word per key pair (0xFFFF per
+      // kept half: masked keys and keys past Nk turn into bf16 -inf in the
+      // bias).  B: -lse*log2(e) and -Delta of the query columns (columns past
+      // Nq get -lse = -inf, so P = 0 there).
+      float *rv = reinterpret_cast<float *>(smem + L::kOffRowv) + (it & 1) * 2 * kBwdTile;
       if (!kB) {
-        const int k0 = o0 + 4 * lane;
+        if (t < kBwdTile / 2) {
+          uint32_t keep = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          keepw[e] = __ballot_sync(0xffffffffu, k0 + e < p.Nk && (mrow == nullptr || mrow[k0 + e] != 0));
+          for (int e = 0; e < 2; ++e) {
+            const int key = o0 + 2 * t + e;
+            if (key < p.Nk && (mrow == nullptr || mrow[key] != 0)) keep |= 0xFFFFu << (16 * e);
+          }
+          reinterpret_cast<uint32_t *>(rv)[t] = keep;
+        }
       } else {
         const int qi = o0 + t;
         const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
-        float *wv = const_cast<float *>(rv);
-        wv[t] = qi < p.Nq ? p.lse[at] * l2e : INFINITY;  // +inf: column past Nq (P = 0)
-        wv[kBwdTile + t] = qi < p.Nq ? p.delta[at] : 0.f;
+        const float lse = qi < p.Nq ? p.lse[at] : 0.f;
+        rv[t] = qi >= p.Nq ? -INFINITY : (lse == -INFINITY ? 0.f : -lse * l2e);  // see the A side
+        rv[kBwdTile + t] = qi < p.Nq ? -p.delta[at] : 0.f;
       }
       ok = named_bar_and(1, kBwdTile, ok);
       if (!ok) break;
       tc_fence_after_sync();
-      // two halves of 64 columns: S, dP -> P, dS
+      const float2 cs2 = make_float2(c_s, c_s), l2e2 = make_float2(l2e, l2e);
+      // A: this row's -lse and -Delta; B: a masked key row gets -inf exponents
+      const float2 rowl2 = make_float2(-lse2, -lse2), rowd2 = make_float2(-delta, -delta);
+      const float kill = key_ok ? 0.f : -INFINITY;
+      const float2 kill2 = make_float2(kill, kill);
+      // two halves of 64 columns: S, dP -> P, dS, two columns per packed op
 #pragma unroll 1
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t sv[64], dpv[64];
@@ -319,54 +333,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
         uint32_t pk[32], dk[32];
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
-          // eight columns: bias values and the column terms
-          float bv[8], l2v[8], dlv[8];
-          bool valid[8];
+          const int c = hf * 64 + c8 * 8;  // first of eight columns
+          float2 b2[4], nl2[4], nd2[4];
           if (!kB) {
-            // 128-byte swizzled [query][key] tile: keys 8 c8 .. of row t
-            const int c = hf * 64 + c8 * 8, box = c >> 6, chunk = (c & 63) >> 3;
+            // 128-byte swizzled [query][key] tile: keys c .. c+7 of row t,
+            // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
+            const int box = c >> 6, chunk = (c & 63) >> 3;
             const uint4 w4 = *reinterpret_cast<const uint4 *>(bt + box * (L::kBiasBytes / 2) + t * 128 +
                                                               ((chunk ^ (t & 7)) << 4));
-            const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+            const uint4 k4 = reinterpret_cast<const uint4 *>(rv)[c8 + hf * 8];
+            const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              bv[e] = (e & 1) ? bf16hi_to_f32(ww[e >> 1]) : bf16lo_to_f32(ww[e >> 1]);
-              const int cc = c + e;
-              valid[e] = ((keepw[cc & 3] >> (cc >> 2)) & 1u) && r < p.Nq;
-              l2v[e] = lse2;
-              dlv[e] = delta;
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t w = (ww[e] & kw[e]) | (~kw[e] & 0xFF80FF80u);
+              b2[e] = make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+              nl2[e] = rowl2;
+              nd2[e] = rowd2;
             }
           } else {
-            // plain [query][key] tile: queries 8 c8 .. of key column t
-            const int c = hf * 64 + c8 * 8;
+            // plain [query][key] tile: queries c .. c+7 of key column t
             const float4 la = *reinterpret_cast<const float4 *>(rv + c), lb = *reinterpret_cast<const float4 *>(rv + c + 4);
             const float4 da = *reinterpret_cast<const float4 *>(rv + kBwdTile + c);
             const float4 db = *reinterpret_cast<const float4 *>(rv + kBwdTile + c + 4);
-            const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-            const float dv8[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+            const float2 lv[4] = {make_float2(la.x, la.y), make_float2(la.z, la.w), make_float2(lb.x, lb.y),
+                                  make_float2(lb.z, lb.w)};
+            const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w), make_float2(db.x, db.y),
+                                  make_float2(db.z, db.w)};
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              bv[e] = __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t *>(bt + (c + e) * 256 + t * 2)) << 16);
-              valid[e] = key_ok;  // columns past Nq carry lse = +inf, so P = 0 there
-              l2v[e] = lv[e];
-              dlv[e] = dv8[e];
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t b0 = *reinterpret_cast<const uint16_t *>(bt + (c + 2 * e) * 256 + t * 2);
+              const uint32_t b1 = *reinterpret_cast<const uint16_t *>(bt + (c + 2 * e + 1) * 256 + t * 2);
+              b2[e] = make_float2(__uint_as_float(b0 << 16), __uint_as_float(b1 << 16));
+              nl2[e] = fadd2(lv[e], kill2);
+              nd2[e] = dv[e];
             }
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int ee = c8 * 8 + e;
-            float pe = 0.f, ds = 0.f;
-            if (valid[e] && bv[e] != -INFINITY) {
-              pe = ex2_approx(fmaf(__uint_as_float(sv[ee]), c_s, fmaf(bv[e], l2e, -l2v[e])));
-              ds = pe * (__uint_as_float(dpv[ee]) - dlv[e]);
-            }
-            if (e & 1) {
-              pk[ee >> 1] |= pack_bf16x2(0.f, pe) & 0xFFFF0000u;
-              dk[ee >> 1] |= pack_bf16x2(0.f, ds) & 0xFFFF0000u;
-            } else {
-              pk[ee >> 1] = pack_bf16x2(pe, 0.f) & 0xFFFFu;
-              dk[ee >> 1] = pack_bf16x2(ds, 0.f) & 0xFFFFu;
-            }
+          for (int e = 0; e < 4; ++e) {
+            const int j = c8 * 4 + e;  // column pair
+            // log2 of P: (tau s + b - lse) log2(e); -inf for masked keys and -inf bias
+            const float2 a = ffma2(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), cs2,
+                                   ffma2(b2[e], l2e2, nl2[e]));
+            const float2 pe = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+            const float2 ds = fmul2(pe, fadd2(make_float2(__uint_as_float(dpv[2 * j]), __uint_as_float(dpv[2 * j + 1])),
+                                              nd2[e]));
+            pk[j] = pack_bf16x2(pe.x, pe.y);
+            dk[j] = pack_bf16x2(ds.x, ds.y);
           }
         }
         if (!kB) {
