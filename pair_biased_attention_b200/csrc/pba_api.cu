@@ -395,11 +395,11 @@ cudaError_t launch_pwa(const pba::PwaParams &p, int grid, cudaStream_t stream) {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
     cudaFuncAttributes fa;
     if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
-        fa.numRegs * pba::kAttnThreads < pba::kRegSplitTotal)
+        fa.numRegs * pba::kPwaThreads < pba::kPwaRegSplitTotal)
       attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
-  kern<<<grid, pba::kAttnThreads, L::kSmemAlloc, stream>>>(p);
+  kern<<<grid, pba::kPwaThreads, L::kSmemAlloc, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -610,7 +610,7 @@ pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v
     // v [S][N][H][D] as (D, N, H, S)
     const uint64_t dims[4] = {uint64_t(D), uint64_t(N), uint64_t(H), uint64_t(S)};
     const int64_t st[3] = {H * D * 2, D * 2, N * H * D * 2};
-    const uint32_t box[4] = {uint32_t(D), uint32_t(pba::kBN), 1, uint32_t(slabs)};
+    const uint32_t box[4] = {uint32_t(D), uint32_t(pba::kPwaBN), 1, uint32_t(slabs)};
     if (!make_map(&p.tm_v, v, dims, st, box, D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return PBA_ERR_INVALID_ARG;
   }
@@ -618,18 +618,18 @@ pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v
     // bias [H][N][N] as (keys, rows, H, 1): two 64-key boxes per tile
     const uint64_t dims[4] = {uint64_t(N), uint64_t(N), uint64_t(H), 1};
     const int64_t st[3] = {N * 2, N * N * 2, 0};
-    const uint32_t box[4] = {64, uint32_t(pba::kBM), 1, 1};
+    const uint32_t box[4] = {64, uint32_t(pba::kPwaBM), 1, 1};
     if (!make_map(&p.tm_bias, bias, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
   }
   p.S = int(S);
   p.N = int(N);
   p.H = int(H);
-  p.n_qblocks = int((N + pba::kQTiles * pba::kBM - 1) / (pba::kQTiles * pba::kBM));
+  p.n_qblocks = int((N + pba::kPwaQTiles * pba::kPwaBM - 1) / (pba::kPwaQTiles * pba::kPwaBM));
   p.n_ftiles = int((S + slabs - 1) / slabs);
   const int64_t n_units = int64_t(H) * p.n_qblocks * p.n_ftiles;
   if (n_units > kMaxI32) return PBA_ERR_INVALID_ARG;
   p.n_units = int(n_units);
-  p.masked = (key_mask != nullptr) || (N % pba::kBN != 0);
+  p.masked = (key_mask != nullptr) || (N % pba::kPwaBN != 0);
   p.mask_vec4 = key_mask != nullptr && (reinterpret_cast<uintptr_t>(key_mask) & 3u) == 0;
   p.mask = key_mask;
   p.out = static_cast<uint16_t *>(out);

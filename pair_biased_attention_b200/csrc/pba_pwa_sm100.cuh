@@ -36,6 +36,21 @@
 
 namespace pba {
 
+// Tile shape, warp roles and register split of this kernel (the same
+// arrangement as the attention kernel's two-warpgroup form).
+constexpr int kPwaBM = 128;           // query rows per tile
+constexpr int kPwaBN = 128;           // keys per tile
+constexpr int kPwaQTiles = 2;         // query tiles per unit
+constexpr int kPwaBiasStages = 2;
+constexpr int kPwaThreads = 384;      // 12 warps
+constexpr int kPwaWarpProducer = 8;
+constexpr int kPwaWarpMma = 9;
+constexpr int kPwaWarpBiasProducer = 11;
+constexpr uint32_t kPwaTmemCols = 512;
+constexpr int kPwaRegsSoftmax = 224;
+constexpr int kPwaRegsOther = 56;
+constexpr int kPwaRegSplitTotal = 256 * kPwaRegsSoftmax + 128 * kPwaRegsOther;
+
 struct PwaParams {
   CUtensorMap tm_v;     // v [S][N][H][D] as (D, N, H, S), box {D, 128, 1, kSlabs}
   CUtensorMap tm_bias;  // bias [H][N][N] as (N keys, N rows, H, 1), box {64, 128, 1, 1}
@@ -61,31 +76,31 @@ struct PwaLayout {
   static constexpr int kRowBytes = D * 2;
   static constexpr int kSwizzleMode = (D == 64) ? 2 : 4;  // 128-byte / 64-byte swizzle
   static constexpr int kAtomBytes = 8 * kRowBytes;        // 8 key rows
-  static constexpr int kSlabBytes = kBN * kRowBytes;      // one sequence's [128 keys][D]
+  static constexpr int kSlabBytes = kPwaBN * kRowBytes;      // one sequence's [128 keys][D]
   static constexpr int kVBytes = kSlabs * kSlabBytes;
   static constexpr int kVStages = 2;
-  static constexpr int kBiasBytes = kBM * kBN * 2;
-  static constexpr int kBiasSlots = kQTiles * kBiasStages;
+  static constexpr int kBiasBytes = kPwaBM * kPwaBN * 2;
+  static constexpr int kBiasSlots = kPwaQTiles * kPwaBiasStages;
   static constexpr int kOffV = 0;
   static constexpr int kOffBias = kOffV + kVStages * kVBytes;
   static constexpr int kOffMaskWords = kOffBias + kBiasSlots * kBiasBytes;
-  static constexpr int kOffBar = kOffMaskWords + kBiasSlots * (kBN / 2) * 4;
+  static constexpr int kOffBar = kOffMaskWords + kBiasSlots * (kPwaBN / 2) * 4;
   static constexpr int kBarVFull = 0;
   static constexpr int kBarVEmpty = kBarVFull + kVStages;
   static constexpr int kBarBiasFull = kBarVEmpty + kVStages;
   static constexpr int kBarBiasReady = kBarBiasFull + kBiasSlots;
   static constexpr int kBarBiasEmpty = kBarBiasReady + kBiasSlots;
   static constexpr int kBarPFull = kBarBiasEmpty + kBiasSlots;  // [w]
-  static constexpr int kBarODone = kBarPFull + kQTiles;
-  static constexpr int kBarOFree = kBarODone + kQTiles;
-  static constexpr int kBarDrain = kBarOFree + kQTiles;
+  static constexpr int kBarODone = kBarPFull + kPwaQTiles;
+  static constexpr int kBarOFree = kBarODone + kPwaQTiles;
+  static constexpr int kBarDrain = kBarOFree + kPwaQTiles;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemSlot + 4;
   static constexpr int kBytes = kOffAbort + 4;
   static constexpr int kSmemAlloc = kBytes + 1024;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
-  static_assert(2 * 64 + kQTiles * kDF <= 512, "Tensor Memory budget");
+  static_assert(2 * 64 + kPwaQTiles * kDF <= 512, "Tensor Memory budget");
 };
 
 struct PwaUnit {
@@ -94,11 +109,11 @@ struct PwaUnit {
 __device__ __forceinline__ PwaUnit decode_pwa_unit(const PwaParams &p, int u) {
   const int f = u % p.n_ftiles;
   const int r = u / p.n_ftiles;
-  return PwaUnit{r / p.n_qblocks, (r % p.n_qblocks) * (kQTiles * kBM), f};
+  return PwaUnit{r / p.n_qblocks, (r % p.n_qblocks) * (kPwaQTiles * kPwaBM), f};
 }
 
 template <int D, bool kGate, bool kMasked>
-__global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __grid_constant__ PwaParams p) {
+__global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __grid_constant__ PwaParams p) {
   using L = PwaLayout<D>;
   constexpr int kExpEmuEvery = (D == 32) ? PBA_EXP_EMU_EVERY_D32 : PBA_EXP_EMU_EVERY_D64;
   extern __shared__ uint8_t smem_raw[];
@@ -109,7 +124,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nt = (p.N + kBN - 1) / kBN;  // key tiles per unit
+  const int nt = (p.N + kPwaBN - 1) / kPwaBN;  // key tiles per unit
   const int u_begin = blockIdx.x, u_step = gridDim.x;
 
   if (threadIdx.x == 0) {
@@ -120,23 +135,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
     for (int i = 0; i < L::kBiasSlots; ++i) {
       mbar_init(&bars[L::kBarBiasFull + i], 1);
       mbar_init(&bars[L::kBarBiasReady + i], 32);
-      mbar_init(&bars[L::kBarBiasEmpty + i], kBM);
+      mbar_init(&bars[L::kBarBiasEmpty + i], kPwaBM);
     }
-    for (int w = 0; w < kQTiles; ++w) {
-      mbar_init(&bars[L::kBarPFull + w], kBM);
+    for (int w = 0; w < kPwaQTiles; ++w) {
+      mbar_init(&bars[L::kBarPFull + w], kPwaBM);
       mbar_init(&bars[L::kBarODone + w], 1);
-      mbar_init(&bars[L::kBarOFree + w], kBM);
+      mbar_init(&bars[L::kBarOFree + w], kPwaBM);
     }
     mbar_init(&bars[L::kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kWarpMma) {
-    tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == kPwaWarpMma) {
+    tmem_alloc(tmem_slot, kPwaTmemCols);
     tmem_relinquish();
   }
-  if (warp == kWarpProducer && lane == 0) tma_prefetch_desc(&p.tm_v);
-  if (warp == kWarpBiasProducer && lane == 0) tma_prefetch_desc(&p.tm_bias);
+  if (warp == kPwaWarpProducer && lane == 0) tma_prefetch_desc(&p.tm_v);
+  if (warp == kPwaWarpBiasProducer && lane == 0) tma_prefetch_desc(&p.tm_bias);
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -147,8 +162,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
   wc_drain.abort_flag = &drain_abort;
 
   if (warp >= 8) {
-    setmaxnreg_dec<kRegsOther>();
-    if (warp == kWarpProducer) {
+    setmaxnreg_dec<kPwaRegsOther>();
+    if (warp == kPwaWarpProducer) {
       // ============================================================== value tiles
       if (lane == 0) {
         const uint64_t pol_keep = l2_policy_evict_last();  // re-read by the other query blocks
@@ -162,7 +177,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
             if (!ok) break;
             mbar_arrive_expect_tx(&bars[L::kBarVFull + s], L::kVBytes);
             // [kSlabs sequences][128 keys][D]; sequences past S read as zero
-            tma_load_4d(smem + L::kOffV + s * L::kVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kBN, un.h,
+            tma_load_4d(smem + L::kOffV + s * L::kVBytes, &p.tm_v, &bars[L::kBarVFull + s], 0, j * kPwaBN, un.h,
                         un.f * L::kSlabs, pol_keep);
             ++vc;
           }
@@ -173,7 +188,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
             if (a > 0) mbar_wait(&bars[L::kBarVFull + s], (a - 1) & 1, wc_drain);
           }
       }
-    } else if (warp == kWarpBiasProducer) {
+    } else if (warp == kPwaWarpBiasProducer) {
       // ============================================================== bias tiles
       if (lane == 0) {
         const uint64_t pol = l2_policy_evict_last();  // shared by the feature tiles of a row block
@@ -182,33 +197,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
         for (int u = u_begin; u < p.n_units && ok; u += u_step) {
           const PwaUnit un = decode_pwa_unit(p, u);
           for (int j = 0; j < nt && ok; ++j, ++gt) {
-            const int t = gt % kBiasStages;
-            for (int w = 0; w < kQTiles && ok; ++w) {
-              const int slot = w * kBiasStages + t;
-              if (gt >= kBiasStages)
-                ok = mbar_wait(&bars[L::kBarBiasEmpty + slot], ((gt / kBiasStages) - 1) & 1, wc);
+            const int t = gt % kPwaBiasStages;
+            for (int w = 0; w < kPwaQTiles && ok; ++w) {
+              const int slot = w * kPwaBiasStages + t;
+              if (gt >= kPwaBiasStages)
+                ok = mbar_wait(&bars[L::kBarBiasEmpty + slot], ((gt / kPwaBiasStages) - 1) & 1, wc);
               if (!ok) break;
               uint8_t *dst = smem + L::kOffBias + slot * L::kBiasBytes;
               mbar_arrive_expect_tx(&bars[L::kBarBiasFull + slot], L::kBiasBytes);
-              tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN, un.q0 + w * kBM, un.h, 0, pol);
-              tma_load_4d(dst + L::kBiasBytes / 2, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kBN + 64,
-                          un.q0 + w * kBM, un.h, 0, pol);
+              tma_load_4d(dst, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kPwaBN, un.q0 + w * kPwaBM, un.h, 0, pol);
+              tma_load_4d(dst + L::kBiasBytes / 2, &p.tm_bias, &bars[L::kBarBiasFull + slot], j * kPwaBN + 64,
+                          un.q0 + w * kPwaBM, un.h, 0, pol);
               ++issued;
             }
           }
         }
         if (!ok)
-          for (int w = 0; w < kQTiles; ++w)
-            for (int t = 0; t < kBiasStages; ++t) {
-              const int n_w = issued / kQTiles + (w < issued % kQTiles ? 1 : 0);
-              const int a = (n_w - t + kBiasStages - 1) / kBiasStages;
-              if (a > 0) mbar_wait(&bars[L::kBarBiasFull + w * kBiasStages + t], (a - 1) & 1, wc_drain);
+          for (int w = 0; w < kPwaQTiles; ++w)
+            for (int t = 0; t < kPwaBiasStages; ++t) {
+              const int n_w = issued / kPwaQTiles + (w < issued % kPwaQTiles ? 1 : 0);
+              const int a = (n_w - t + kPwaBiasStages - 1) / kPwaBiasStages;
+              if (a > 0) mbar_wait(&bars[L::kBarBiasFull + w * kPwaBiasStages + t], (a - 1) & 1, wc_drain);
             }
       }
-    } else if (warp == kWarpMma) {
+    } else if (warp == kPwaWarpMma) {
       // ============================================================== P V MMAs
       if (lane == 0) {
-        const uint32_t idesc = idesc_bf16_f32(kBM, L::kDF, true);  // V is MN-major
+        const uint32_t idesc = idesc_bf16_f32(kPwaBM, L::kDF, true);  // V is MN-major
         const uint32_t sV = smem_u32(smem + L::kOffV);
         constexpr uint32_t kDescHi = smem_desc_hi(L::kAtomBytes, L::kSwizzleMode);
         bool ok = true;
@@ -217,7 +232,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
           for (int j = 0; j < nt && ok; ++j) {
             const int s = vc % L::kVStages;
             ok = mbar_wait(&bars[L::kBarVFull + s], (vc / L::kVStages) & 1, wc);
-            for (int w = 0; w < kQTiles && ok; ++w) {
+            for (int w = 0; w < kPwaQTiles && ok; ++w) {
               if (!(ok = mbar_wait(&bars[L::kBarPFull + w], gp & 1, wc))) break;
               // the first P V of a unit overwrites O: the epilogue must have read it
               if (j == 0 && uc > 0 && !(ok = mbar_wait(&bars[L::kBarOFree + w], (uc - 1) & 1, wc))) break;
@@ -227,7 +242,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
               // B: keys 16 kk .. 16 kk + 15 of every slab (slabs LBO apart)
               const uint32_t v_lo = smem_desc_lo(sV + s * L::kVBytes, L::kSlabBytes);
 #pragma unroll 4
-              for (int kk = 0; kk < kBN / 16; ++kk)
+              for (int kk = 0; kk < kPwaBN / 16; ++kk)
                 mma_bf16_ts(d_tmem, a_tmem + kk * 8, desc_join(v_lo + kk * (16 * L::kRowBytes / 16), kDescHi), idesc,
                             (j > 0 || kk > 0) ? 1u : 0u);
               tc_commit(&bars[L::kBarODone + w]);
@@ -249,7 +264,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
       int gt = 0;
       for (int u = u_begin; u < p.n_units && ok; u += u_step) {
         auto load_word = [&](int j) -> uint32_t {  // byte e nonzero = key 4*lane+e takes part
-          const int key0 = j * kBN + 4 * lane;
+          const int key0 = j * kPwaBN + 4 * lane;
           if (p.mask == nullptr) return 0x01010101u;
           if (p.mask_vec4 && key0 + 3 < p.N) return __ldg(reinterpret_cast<const uint32_t *>(p.mask + key0));
           uint32_t wv = 0;
@@ -262,19 +277,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
         for (int j = 0; j < nt && ok; ++j, ++gt) {
           const uint32_t word = next_word;
           if (j + 1 < nt) next_word = load_word(j + 1);
-          const int key0 = j * kBN + 4 * lane;
+          const int key0 = j * kPwaBN + 4 * lane;
           uint32_t inv = 0;
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             if (key0 + e >= p.N || ((word >> (8 * e)) & 0xFFu) == 0) inv |= 1u << e;
           const uint2 keep = make_uint2(((inv & 1u) ? 0u : 0x0000FFFFu) | ((inv & 2u) ? 0u : 0xFFFF0000u),
                                         ((inv & 4u) ? 0u : 0x0000FFFFu) | ((inv & 8u) ? 0u : 0xFFFF0000u));
-          const int t = gt % kBiasStages;
-          for (int w = 0; w < kQTiles && ok; ++w) {
-            const int slot = w * kBiasStages + t;
-            ok = mbar_wait<false>(&bars[L::kBarBiasFull + slot], (gt / kBiasStages) & 1, wc);
+          const int t = gt % kPwaBiasStages;
+          for (int w = 0; w < kPwaQTiles && ok; ++w) {
+            const int slot = w * kPwaBiasStages + t;
+            ok = mbar_wait<false>(&bars[L::kBarBiasFull + slot], (gt / kPwaBiasStages) & 1, wc);
             if (!ok) break;
-            reinterpret_cast<uint2 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[lane] = keep;
+            reinterpret_cast<uint2 *>(smem + L::kOffMaskWords + slot * (kPwaBN / 2) * 4)[lane] = keep;
             __syncwarp();
             mbar_arrive(&bars[L::kBarBiasReady + slot]);
           }
@@ -283,7 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
     }
   } else {
     // ================================================================ softmax warpgroups
-    setmaxnreg_inc<kRegsSoftmax>();
+    setmaxnreg_inc<kPwaRegsSoftmax>();
     const int w = warp >> 2;
     const int t = threadIdx.x & 127;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
@@ -295,21 +310,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
       float m_cur = -INFINITY;  // maximum used for P and l
       float l = 0.f;
       for (int j = 0; j < nt && ok; ++j, ++gt) {
-        const int slot = w * kBiasStages + (gt % kBiasStages);
-        ok = mbar_wait<false>(&bars[(kMasked ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1,
+        const int slot = w * kPwaBiasStages + (gt % kPwaBiasStages);
+        ok = mbar_wait<false>(&bars[(kMasked ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kPwaBiasStages) & 1,
                               wc);
         if (!ok) break;
         const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
         // the logits of this row's 128 keys (masked ones -inf)
-        float2 x[kBN / 2];
+        float2 x[kPwaBN / 2];
 #pragma unroll
-        for (int c8 = 0; c8 < kBN / 8; ++c8) {
+        for (int c8 = 0; c8 < kPwaBN / 8; ++c8) {
           const int box = c8 >> 3, chunk = c8 & 7;
           const uint4 bv =
               *reinterpret_cast<const uint4 *>(tile + box * (L::kBiasBytes / 2) + t * 128 + ((chunk ^ (t & 7)) << 4));
           uint32_t wv[4] = {bv.x, bv.y, bv.z, bv.w};
           if (kMasked) {
-            const uint4 kv = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kBN / 2) * 4)[c8];
+            const uint4 kv = reinterpret_cast<const uint4 *>(smem + L::kOffMaskWords + slot * (kPwaBN / 2) * 4)[c8];
             const uint32_t keep[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) wv[e] = (wv[e] & keep[e]) | (~keep[e] & 0xFF80FF80u);
@@ -323,7 +338,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = fmaxf(x[i].x, x[i].y);
 #pragma unroll
-        for (int i = 8; i < kBN / 2; ++i) m8[i & 7] = max3f(m8[i & 7], x[i].x, x[i].y);
+        for (int i = 8; i < kPwaBN / 2; ++i) m8[i & 7] = max3f(m8[i & 7], x[i].x, x[i].y);
         const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         const bool need = mx > m_cur + kRescaleThreshold;
         float alpha = 1.f;
@@ -334,10 +349,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
         }
         const float neg_m = (m_cur == -INFINITY) ? 0.f : -m_cur * kLog2e;
         const float2 l2e2 = make_float2(kLog2e, kLog2e), negm2 = make_float2(neg_m, neg_m);
-        uint32_t pk[kBN / 2];
+        uint32_t pk[kPwaBN / 2];
         float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int i = 0; i < kBN / 2; ++i) {
+        for (int i = 0; i < kPwaBN / 2; ++i) {
           const float2 a = ffma2(x[i], l2e2, negm2);
           const float2 pv = (kExpEmuEvery > 0 && i % kExpEmuEvery == kExpEmuEvery - 1)
                                 ? exp2_poly2(a)
@@ -366,7 +381,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
           }
         }
 #pragma unroll
-        for (int c = 0; c < kBN / 2; c += 32) tmem_st32(tP + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
+        for (int c = 0; c < kPwaBN / 2; c += 32) tmem_st32(tP + c, *reinterpret_cast<uint32_t(*)[32]>(&pk[c]));
         tmem_wait_st();
         tc_fence_before_sync();
         mbar_arrive(&bars[L::kBarPFull + w]);
@@ -377,7 +392,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
       if (!ok) break;
       tc_fence_after_sync();
       const PwaUnit un = decode_pwa_unit(p, u);
-      const int row = un.q0 + w * kBM + t;
+      const int row = un.q0 + w * kPwaBM + t;
       const bool live = row < p.N;
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
@@ -424,7 +439,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_pwa_sm100_kernel(const __
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kPwaWarpMma) tmem_dealloc(tmem, kPwaTmemCols);
 }
 
 }  // namespace pba
