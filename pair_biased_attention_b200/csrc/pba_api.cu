@@ -419,6 +419,11 @@ cudaError_t launch_bwd(const pba::BwdParams &p, int grid, cudaStream_t stream) {
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+    // the register split must fit in what the block is launched with (see launch_tc)
+    cudaFuncAttributes fa;
+    if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+        fa.numRegs * pba::kBwdThreads < pba::kBwdRegSplitTotal)
+      attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kBwdThreads, L::kSmemAlloc, stream>>>(p);

@@ -19,12 +19,12 @@
 // Tensor Memory and dO, Q read MN-major.  Both recompute P from the saved
 // log-sum-exp, so no N^2 intermediate is stored besides dbias.
 //
-// One CTA per unit, 192 threads: warps 0-3 the compute warpgroup (row =
-// thread = Tensor Memory lane), warp 4 the TMA producer, warp 5 Tensor Memory
-// and the MMAs.  Per step the chain is S, dP -> P, dS -> dQ or dV, dK; the
-// next step's S, dP are issued as soon as this step's have been read, so they
-// overlap the second half of the elementwise work.  Operand tiles are
-// double-buffered.
+// One CTA per unit, 384 threads: warps 0-7 two compute warpgroups (row =
+// thread = Tensor Memory lane; warpgroup g takes columns 64g .. 64g+63 of
+// every step), warp 8 the TMA producer, warp 9 Tensor Memory and the MMAs,
+// warps 10-11 idle.  Per step the chain is S, dP -> P, dS -> dQ or dV, dK; the
+// next step's S, dP are issued as soon as both warpgroups have read this
+// step's.  Operand tiles are double-buffered.
 #pragma once
 
 #include <cuda.h>
@@ -34,8 +34,17 @@
 
 namespace pba {
 
-constexpr int kBwdThreads = 192;
 constexpr int kBwdTile = 128;
+constexpr int kBwdComputeGroups = 2;  // column halves of a step, one warpgroup each
+constexpr int kBwdThreads = 128 * (kBwdComputeGroups + 1);
+constexpr int kBwdWarpProducer = 4 * kBwdComputeGroups;
+constexpr int kBwdWarpMma = kBwdWarpProducer + 1;
+// Per-thread register limits after the warpgroup reallocation: the launch
+// gives 168 (384 x 168 = 64512); the producer/MMA warpgroup keeps 56 and the
+// compute warpgroups take 224 (128 x 56 + 256 x 224 = 64512).
+constexpr int kBwdRegsCompute = 224;
+constexpr int kBwdRegsOther = 56;
+constexpr int kBwdRegSplitTotal = 128 * kBwdComputeGroups * kBwdRegsCompute + 128 * kBwdRegsOther;
 
 struct BwdParams {
   // A: tm_q/tm_do are the query-side tiles, tm_k/tm_v the key-side tiles;
@@ -123,17 +132,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     mbar_init(&bars[L::kBarFixFull], 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[L::kBarStepFull + s], 1);
-      mbar_init(&bars[L::kBarStepEmpty + s], 2);  // the MMA commit + the compute warpgroup (bias, row values)
+      // the MMA commit + each compute warpgroup (bias, row values)
+      mbar_init(&bars[L::kBarStepEmpty + s], 1 + kBwdComputeGroups);
     }
     mbar_init(&bars[L::kBarSFull], 1);
-    mbar_init(&bars[L::kBarSFree], kBwdTile);
-    mbar_init(&bars[L::kBarGFull], kBwdTile);
+    mbar_init(&bars[L::kBarSFree], kBwdComputeGroups * kBwdTile);
+    mbar_init(&bars[L::kBarGFull], kBwdComputeGroups * kBwdTile);
     mbar_init(&bars[L::kBarGDone], 1);
     mbar_init(&bars[L::kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kBwdWarpMma) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -146,114 +156,119 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
   int drain_abort = 0;
   wc_drain.abort_flag = &drain_abort;
 
-  if (warp == 4) {
-    // ================================================================ TMA producer
-    if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_last();
-      // fixed tiles of the unit: A: Q, dO rows; B: K, V rows
-      mbar_arrive_expect_tx(&bars[L::kBarFixFull], 2 * L::kTileBytes);
-      tma_load_4d(smem + L::kOffFix0, kB ? &p.tm_k : &p.tm_q, &bars[L::kBarFixFull], 0, row0, h, b, pol);
-      tma_load_4d(smem + L::kOffFix1, kB ? &p.tm_v : &p.tm_do, &bars[L::kBarFixFull], 0, row0, h, b, pol);
-      bool ok = true;
-      int it = 0;
-      for (; it < nsteps && ok; ++it) {
-        const int s = it % L::kStages;
-        if (it >= L::kStages) ok = mbar_wait(&bars[L::kBarStepEmpty + s], ((it / L::kStages) - 1) & 1, wc);
-        if (!ok) break;
-        const int o0 = it * kBwdTile;
-        uint64_t *full = &bars[L::kBarStepFull + s];
-        mbar_arrive_expect_tx(full, 2 * L::kTileBytes + L::kBiasBytes);
-        tma_load_4d(smem + L::kOffStep0 + s * L::kTileBytes, kB ? &p.tm_q : &p.tm_k, full, 0, o0, h, b, pol);
-        tma_load_4d(smem + L::kOffStep1 + s * L::kTileBytes, kB ? &p.tm_do : &p.tm_v, full, 0, o0, h, b, pol);
-        uint8_t *bdst = smem + L::kOffBias + s * L::kBiasBytes;
-        const int hb = p.bias_h_bcast ? 0 : h, bb = p.bias_b_bcast ? 0 : b;
-        if (kB) {
-          // [128 queries][128 keys], no swizzle: the thread of key j reads column j
-          tma_load_4d(bdst, &p.tm_bias, full, row0, o0, hb, bb, pol);
-        } else {
-          // [128 queries][128 keys] as two 64-key boxes, 128-byte swizzle
-          tma_load_4d(bdst, &p.tm_bias, full, o0, row0, hb, bb, pol);
-          tma_load_4d(bdst + L::kBiasBytes / 2, &p.tm_bias, full, o0 + 64, row0, hb, bb, pol);
+  if (warp >= kBwdWarpProducer) {
+    setmaxnreg_dec<kBwdRegsOther>();
+    if (warp == kBwdWarpProducer) {
+      // ================================================================ TMA producer
+      if (lane == 0) {
+        const uint64_t pol = l2_policy_evict_last();
+        // fixed tiles of the unit: A: Q, dO rows; B: K, V rows
+        mbar_arrive_expect_tx(&bars[L::kBarFixFull], 2 * L::kTileBytes);
+        tma_load_4d(smem + L::kOffFix0, kB ? &p.tm_k : &p.tm_q, &bars[L::kBarFixFull], 0, row0, h, b, pol);
+        tma_load_4d(smem + L::kOffFix1, kB ? &p.tm_v : &p.tm_do, &bars[L::kBarFixFull], 0, row0, h, b, pol);
+        bool ok = true;
+        int it = 0;
+        for (; it < nsteps && ok; ++it) {
+          const int s = it % L::kStages;
+          if (it >= L::kStages) ok = mbar_wait(&bars[L::kBarStepEmpty + s], ((it / L::kStages) - 1) & 1, wc);
+          if (!ok) break;
+          const int o0 = it * kBwdTile;
+          uint64_t *full = &bars[L::kBarStepFull + s];
+          mbar_arrive_expect_tx(full, 2 * L::kTileBytes + L::kBiasBytes);
+          tma_load_4d(smem + L::kOffStep0 + s * L::kTileBytes, kB ? &p.tm_q : &p.tm_k, full, 0, o0, h, b, pol);
+          tma_load_4d(smem + L::kOffStep1 + s * L::kTileBytes, kB ? &p.tm_do : &p.tm_v, full, 0, o0, h, b, pol);
+          uint8_t *bdst = smem + L::kOffBias + s * L::kBiasBytes;
+          const int hb = p.bias_h_bcast ? 0 : h, bb = p.bias_b_bcast ? 0 : b;
+          if (kB) {
+            // [128 queries][128 keys], no swizzle: the thread of key j reads column j
+            tma_load_4d(bdst, &p.tm_bias, full, row0, o0, hb, bb, pol);
+          } else {
+            // [128 queries][128 keys] as two 64-key boxes, 128-byte swizzle
+            tma_load_4d(bdst, &p.tm_bias, full, o0, row0, hb, bb, pol);
+            tma_load_4d(bdst + L::kBiasBytes / 2, &p.tm_bias, full, o0 + 64, row0, hb, bb, pol);
+          }
         }
+        mbar_wait(&bars[L::kBarFixFull], 0, wc_drain);
+        if (!ok)
+          for (int s = 0; s < L::kStages; ++s) {
+            const int a = (it - s + L::kStages - 1) / L::kStages;
+            if (a > 0) mbar_wait(&bars[L::kBarStepFull + s], (a - 1) & 1, wc_drain);
+          }
       }
-      mbar_wait(&bars[L::kBarFixFull], 0, wc_drain);
-      if (!ok)
-        for (int s = 0; s < L::kStages; ++s) {
-          const int a = (it - s + L::kStages - 1) / L::kStages;
-          if (a > 0) mbar_wait(&bars[L::kBarStepFull + s], (a - 1) & 1, wc_drain);
+    } else if (warp == kBwdWarpMma) {
+      // ================================================================ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc_s = idesc_bf16_f32(kBwdTile, kBwdTile, false);  // both operands K-major
+        const uint32_t idesc_g = idesc_bf16_f32(kBwdTile, D, true);          // B MN-major
+        constexpr uint32_t kHi = smem_desc_hi(L::kAtomBytes, L::kSwizzleMode);
+        const uint32_t sF0 = smem_u32(smem + L::kOffFix0), sF1 = smem_u32(smem + L::kOffFix1);
+        // S, dP of step `it` (A: S = Q K^T, dP = dO V^T; B: S^T = K Q^T,
+        // dP^T = V dO^T) once its tiles have landed and the compute warpgroup has
+        // read the previous step's S and dP
+        auto issue_s = [&](int it) -> bool {
+          const int s = it % L::kStages;
+          if (!mbar_wait(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc)) return false;
+          if (it > 0 && !mbar_wait(&bars[L::kBarSFree], (it - 1) & 1, wc)) return false;
+          tc_fence_after_sync();
+          const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
+          const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
+          const uint32_t a0 = smem_desc_lo(sF0, 16), b0 = smem_desc_lo(sS0, 16);
+          const uint32_t a1 = smem_desc_lo(sF1, 16), b1 = smem_desc_lo(sS1, 16);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + L::kColS, desc_join(a0 + kk * 2, kHi), desc_join(b0 + kk * 2, kHi), idesc_s, kk > 0);
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_bf16_ss(tmem + L::kColDP, desc_join(a1 + kk * 2, kHi), desc_join(b1 + kk * 2, kHi), idesc_s, kk > 0);
+          tc_commit(&bars[L::kBarSFull]);
+          return true;
+        };
+        // Software-pipelined: S, dP of step it+1 go out as soon as step it's
+        // S, dP have been read, before the accumulating products of step it.
+        bool ok = mbar_wait(&bars[L::kBarFixFull], 0, wc);
+        if (ok) ok = issue_s(0);
+        for (int it = 0; it < nsteps && ok; ++it) {
+          const int s = it % L::kStages;
+          if (it + 1 < nsteps && !(ok = issue_s(it + 1))) break;
+          // the accumulating products once P / dS are in Tensor Memory
+          ok = mbar_wait(&bars[L::kBarGFull], it & 1, wc);
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
+          const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
+          const uint32_t acc = (it > 0) ? 1u : 0u;
+          if (!kB) {
+            // dQ += dS K: B = the K tile, keys are the reduction (MN-major read)
+            const uint32_t kb = smem_desc_lo(sS0, L::kTileBytes);
+  #pragma unroll
+            for (int kk = 0; kk < kBwdTile / 16; ++kk)
+              mma_bf16_ts(tmem + L::kColAcc0, tmem + L::kColG0 + kk * 8,
+                          desc_join(kb + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
+          } else {
+            // dV += P^T dO and dK += dS^T Q: queries are the reduction
+            const uint32_t qb = smem_desc_lo(sS0, L::kTileBytes), ob = smem_desc_lo(sS1, L::kTileBytes);
+  #pragma unroll
+            for (int kk = 0; kk < kBwdTile / 16; ++kk)
+              mma_bf16_ts(tmem + L::kColAcc1, tmem + L::kColG0 + kk * 8,
+                          desc_join(ob + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
+  #pragma unroll
+            for (int kk = 0; kk < kBwdTile / 16; ++kk)
+              mma_bf16_ts(tmem + L::kColAcc0, tmem + L::kColG1 + kk * 8,
+                          desc_join(qb + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bars[L::kBarGDone]);
+          tc_commit(&bars[L::kBarStepEmpty + s]);
         }
-    }
-  } else if (warp == 5) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kBwdTile, kBwdTile, false);  // both operands K-major
-      const uint32_t idesc_g = idesc_bf16_f32(kBwdTile, D, true);          // B MN-major
-      constexpr uint32_t kHi = smem_desc_hi(L::kAtomBytes, L::kSwizzleMode);
-      const uint32_t sF0 = smem_u32(smem + L::kOffFix0), sF1 = smem_u32(smem + L::kOffFix1);
-      // S, dP of step `it` (A: S = Q K^T, dP = dO V^T; B: S^T = K Q^T,
-      // dP^T = V dO^T) once its tiles have landed and the compute warpgroup has
-      // read the previous step's S and dP
-      auto issue_s = [&](int it) -> bool {
-        const int s = it % L::kStages;
-        if (!mbar_wait(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc)) return false;
-        if (it > 0 && !mbar_wait(&bars[L::kBarSFree], (it - 1) & 1, wc)) return false;
-        tc_fence_after_sync();
-        const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
-        const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
-        const uint32_t a0 = smem_desc_lo(sF0, 16), b0 = smem_desc_lo(sS0, 16);
-        const uint32_t a1 = smem_desc_lo(sF1, 16), b1 = smem_desc_lo(sS1, 16);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + L::kColS, desc_join(a0 + kk * 2, kHi), desc_join(b0 + kk * 2, kHi), idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_bf16_ss(tmem + L::kColDP, desc_join(a1 + kk * 2, kHi), desc_join(b1 + kk * 2, kHi), idesc_s, kk > 0);
-        tc_commit(&bars[L::kBarSFull]);
-        return true;
-      };
-      // Software-pipelined: S, dP of step it+1 go out as soon as step it's
-      // S, dP have been read, before the accumulating products of step it.
-      bool ok = mbar_wait(&bars[L::kBarFixFull], 0, wc);
-      if (ok) ok = issue_s(0);
-      for (int it = 0; it < nsteps && ok; ++it) {
-        const int s = it % L::kStages;
-        if (it + 1 < nsteps && !(ok = issue_s(it + 1))) break;
-        // the accumulating products once P / dS are in Tensor Memory
-        ok = mbar_wait(&bars[L::kBarGFull], it & 1, wc);
-        if (!ok) break;
-        tc_fence_after_sync();
-        const uint32_t sS0 = smem_u32(smem + L::kOffStep0 + s * L::kTileBytes);
-        const uint32_t sS1 = smem_u32(smem + L::kOffStep1 + s * L::kTileBytes);
-        const uint32_t acc = (it > 0) ? 1u : 0u;
-        if (!kB) {
-          // dQ += dS K: B = the K tile, keys are the reduction (MN-major read)
-          const uint32_t kb = smem_desc_lo(sS0, L::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < kBwdTile / 16; ++kk)
-            mma_bf16_ts(tmem + L::kColAcc0, tmem + L::kColG0 + kk * 8,
-                        desc_join(kb + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
-        } else {
-          // dV += P^T dO and dK += dS^T Q: queries are the reduction
-          const uint32_t qb = smem_desc_lo(sS0, L::kTileBytes), ob = smem_desc_lo(sS1, L::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < kBwdTile / 16; ++kk)
-            mma_bf16_ts(tmem + L::kColAcc1, tmem + L::kColG0 + kk * 8,
-                        desc_join(ob + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < kBwdTile / 16; ++kk)
-            mma_bf16_ts(tmem + L::kColAcc0, tmem + L::kColG1 + kk * 8,
-                        desc_join(qb + kk * (16 * L::kRowBytes / 16), kHi), idesc_g, (acc || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bars[L::kBarGDone]);
-        tc_commit(&bars[L::kBarStepEmpty + s]);
+        tc_commit(&bars[L::kBarDrain]);
+        mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
       }
-      tc_commit(&bars[L::kBarDrain]);
-      mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
     }
   } else {
-    // ================================================================ compute warpgroup
-    const int t = threadIdx.x;  // row of the unit's tile = Tensor Memory lane
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    // ================================================================ compute warpgroups
+    setmaxnreg_inc<kBwdRegsCompute>();
+    const int g = warp >> 2;           // column half of each step
+    const int t = threadIdx.x & 127;   // row of the unit's tile = Tensor Memory lane
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const int r = row0 + t;     // A: query row; B: key row
     const float l2e = 1.4426950408889634f;
     const float c_s = p.tau * l2e;
@@ -285,30 +300,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       if (ok && it > 0) ok = mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc);
       const uint8_t *bt = smem + L::kOffBias + s * L::kBiasBytes;
       // Per-step column data in shared memory (double-buffered by step
-      // parity), written by the warpgroup; the barrier also makes the warps
-      // leave the loop together.  A: one keep word per key pair (0xFFFF per
-      // kept half: masked keys and keys past Nk turn into bf16 -inf in the
-      // bias).  B: -lse*log2(e) and -Delta of the query columns (columns past
-      // Nq get -lse = -inf, so P = 0 there).
+      // parity); each warpgroup writes and reads only its own 64 columns, and
+      // its barrier also makes its warps leave the loop together.  A: one
+      // keep word per key pair (0xFFFF per kept half: masked keys and keys
+      // past Nk turn into bf16 -inf in the bias).  B: -lse*log2(e) and -Delta
+      // of the query columns (columns past Nq get -lse = -inf, so P = 0 there).
       float *rv = reinterpret_cast<float *>(smem + L::kOffRowv) + (it & 1) * 2 * kBwdTile;
       if (!kB) {
-        if (t < kBwdTile / 2) {
+        if (t < kBwdTile / 4) {
+          const int pr = g * (kBwdTile / 4) + t;  // key pair of the step
           uint32_t keep = 0;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int key = o0 + 2 * t + e;
+            const int key = o0 + 2 * pr + e;
             if (key < p.Nk && (mrow == nullptr || mrow[key] != 0)) keep |= 0xFFFFu << (16 * e);
           }
-          reinterpret_cast<uint32_t *>(rv)[t] = keep;
+          reinterpret_cast<uint32_t *>(rv)[pr] = keep;
         }
-      } else {
-        const int qi = o0 + t;
+      } else if (t < kBwdTile / 2) {
+        const int col = g * (kBwdTile / 2) + t;  // query column of the step
+        const int qi = o0 + col;
         const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
         const float lse = qi < p.Nq ? p.lse[at] : 0.f;
-        rv[t] = qi >= p.Nq ? -INFINITY : (lse == -INFINITY ? 0.f : -lse * l2e);  // see the A side
-        rv[kBwdTile + t] = qi < p.Nq ? -p.delta[at] : 0.f;
+        rv[col] = qi >= p.Nq ? -INFINITY : (lse == -INFINITY ? 0.f : -lse * l2e);  // see the A side
+        rv[kBwdTile + col] = qi < p.Nq ? -p.delta[at] : 0.f;
       }
-      ok = named_bar_and(1, kBwdTile, ok);
+      ok = named_bar_and(1 + g, kBwdTile, ok);
       if (!ok) break;
       tc_fence_after_sync();
       const float2 cs2 = make_float2(c_s, c_s), l2e2 = make_float2(l2e, l2e);
@@ -316,109 +333,120 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       const float2 rowl2 = make_float2(-lse2, -lse2), rowd2 = make_float2(-delta, -delta);
       const float kill = key_ok ? 0.f : -INFINITY;
       const float2 kill2 = make_float2(kill, kill);
-      // two halves of 64 columns: S, dP -> P, dS, two columns per packed op
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
+      // this warpgroup's 64 columns: S, dP -> P, dS, two columns per packed op
+      {
+        const int hf = g;
         uint32_t sv[64], dpv[64];
         tmem_ld32(tmem + lane_base + L::kColS + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(tmem + lane_base + L::kColS + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_ld32(tmem + lane_base + L::kColDP + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
         tmem_ld32(tmem + lane_base + L::kColDP + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
         tmem_wait_ld();
-        if (hf == 1) {
-          // S and dP are in registers: the next step's S, dP may overwrite them
-          tc_fence_before_sync();
-          mbar_arrive(&bars[L::kBarSFree]);
-        }
-        uint32_t pk[32], dk[32];
+        // S and dP are in registers: the next step's S, dP may overwrite them
+        // once both warpgroups have arrived
+        tc_fence_before_sync();
+        mbar_arrive(&bars[L::kBarSFree]);
+        // two quarters of 32 columns, each stored to Tensor Memory (and, in
+        // A, to dbias) before the next is formed
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const int c = hf * 64 + c8 * 8;  // first of eight columns
-          float2 b2[4], nl2[4], nd2[4];
-          if (!kB) {
-            // 128-byte swizzled [query][key] tile: keys c .. c+7 of row t,
-            // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
-            const int box = c >> 6, chunk = (c & 63) >> 3;
-            const uint4 w4 = *reinterpret_cast<const uint4 *>(bt + box * (L::kBiasBytes / 2) + t * 128 +
-                                                              ((chunk ^ (t & 7)) << 4));
-            const uint4 k4 = reinterpret_cast<const uint4 *>(rv)[c8 + hf * 8];
-            const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
+        for (int qt = 0; qt < 2; ++qt) {
+          uint32_t pk[16], dk[16];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t w = (ww[e] & kw[e]) | (~kw[e] & 0xFF80FF80u);
-              b2[e] = make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
-              nl2[e] = rowl2;
-              nd2[e] = rowd2;
-            }
-          } else {
-            // plain [query][key] tile: queries c .. c+7 of key column t
-            const float4 la = *reinterpret_cast<const float4 *>(rv + c), lb = *reinterpret_cast<const float4 *>(rv + c + 4);
-            const float4 da = *reinterpret_cast<const float4 *>(rv + kBwdTile + c);
-            const float4 db = *reinterpret_cast<const float4 *>(rv + kBwdTile + c + 4);
-            const float2 lv[4] = {make_float2(la.x, la.y), make_float2(la.z, la.w), make_float2(lb.x, lb.y),
-                                  make_float2(lb.z, lb.w)};
-            const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w), make_float2(db.x, db.y),
-                                  make_float2(db.z, db.w)};
+          for (int c8 = 4 * qt; c8 < 4 * qt + 4; ++c8) {
+            const int c = hf * 64 + c8 * 8;  // first of eight columns
+            float2 b2[4], nl2[4], nd2[4];
+            if (!kB) {
+              // 128-byte swizzled [query][key] tile: keys c .. c+7 of row t,
+              // masked halves become bf16 -inf: (w & keep) | (~keep & -inf)
+              const int box = c >> 6, chunk = (c & 63) >> 3;
+              const uint4 w4 = *reinterpret_cast<const uint4 *>(bt + box * (L::kBiasBytes / 2) + t * 128 +
+                                                                ((chunk ^ (t & 7)) << 4));
+              const uint4 k4 = reinterpret_cast<const uint4 *>(rv)[c8 + hf * 8];
+              const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t b0 = *reinterpret_cast<const uint16_t *>(bt + (c + 2 * e) * 256 + t * 2);
-              const uint32_t b1 = *reinterpret_cast<const uint16_t *>(bt + (c + 2 * e + 1) * 256 + t * 2);
-              b2[e] = make_float2(__uint_as_float(b0 << 16), __uint_as_float(b1 << 16));
-              nl2[e] = fadd2(lv[e], kill2);
-              nd2[e] = dv[e];
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = c8 * 4 + e;  // column pair
-            // log2 of P: (tau s + b - lse) log2(e); -inf for masked keys and -inf bias
-            const float2 a = ffma2(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), cs2,
-                                   ffma2(b2[e], l2e2, nl2[e]));
-            const float2 pe = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-            const float2 ds = fmul2(pe, fadd2(make_float2(__uint_as_float(dpv[2 * j]), __uint_as_float(dpv[2 * j + 1])),
-                                              nd2[e]));
-            pk[j] = pack_bf16x2(pe.x, pe.y);
-            dk[j] = pack_bf16x2(ds.x, ds.y);
-          }
-        }
-        if (!kB) {
-          // dbias row segment (64 keys) and dS into Tensor Memory
-          const int key0 = o0 + hf * 64;
-          if (r < p.Nq) {
-            uint16_t *dst = p.dbias + int64_t(b) * p.db_sb + int64_t(h) * p.db_sh + int64_t(r) * p.db_sn + key0;
-            if (key0 + 64 <= p.Nk) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                reinterpret_cast<uint4 *>(dst)[q] = make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t w = (ww[e] & kw[e]) | (~kw[e] & 0xFF80FF80u);
+                b2[e] = make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+                nl2[e] = rowl2;
+                nd2[e] = rowd2;
+              }
             } else {
-              for (int e = 0; key0 + e < p.Nk; ++e) dst[e] = uint16_t((e & 1) ? (dk[e >> 1] >> 16) : (dk[e >> 1] & 0xFFFFu));
+              // plain [query][key] tile: queries c .. c+7 of key column t
+              const float4 la = *reinterpret_cast<const float4 *>(rv + c);
+              const float4 lb = *reinterpret_cast<const float4 *>(rv + c + 4);
+              const float4 da = *reinterpret_cast<const float4 *>(rv + kBwdTile + c);
+              const float4 db = *reinterpret_cast<const float4 *>(rv + kBwdTile + c + 4);
+              const float2 lv[4] = {make_float2(la.x, la.y), make_float2(la.z, la.w), make_float2(lb.x, lb.y),
+                                    make_float2(lb.z, lb.w)};
+              const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w), make_float2(db.x, db.y),
+                                    make_float2(db.z, db.w)};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t b0 = *reinterpret_cast<const uint16_t *>(bt + (c + 2 * e) * 256 + t * 2);
+                const uint32_t b1 = *reinterpret_cast<const uint16_t *>(bt + (c + 2 * e + 1) * 256 + t * 2);
+                b2[e] = make_float2(__uint_as_float(b0 << 16), __uint_as_float(b1 << 16));
+                nl2[e] = fadd2(lv[e], kill2);
+                nd2[e] = dv[e];
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = c8 * 4 + e;  // column pair
+              // log2 of P: (tau s + b - lse) log2(e); -inf for masked keys and -inf bias
+              const float2 a = ffma2(make_float2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1])), cs2,
+                                     ffma2(b2[e], l2e2, nl2[e]));
+              const float2 pe = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+              const float2 dp = make_float2(__uint_as_float(dpv[2 * j]), __uint_as_float(dpv[2 * j + 1]));
+              const float2 ds = fmul2(pe, fadd2(dp, nd2[e]));
+              pk[j - 16 * qt] = pack_bf16x2(pe.x, pe.y);
+              dk[j - 16 * qt] = pack_bf16x2(ds.x, ds.y);
             }
           }
-          tmem_st32(tmem + lane_base + L::kColG0 + hf * 32, dk);
-        } else {
-          tmem_st32(tmem + lane_base + L::kColG0 + hf * 32, pk);  // P^T
-          tmem_st32(tmem + lane_base + L::kColG1 + hf * 32, dk);  // dS^T
+          if (!kB) {
+            // dbias row segment (32 keys) and dS into Tensor Memory
+            const int key0 = o0 + hf * 64 + qt * 32;
+            if (r < p.Nq) {
+              uint16_t *dst = p.dbias + int64_t(b) * p.db_sb + int64_t(h) * p.db_sh + int64_t(r) * p.db_sn + key0;
+              if (key0 + 32 <= p.Nk) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  reinterpret_cast<uint4 *>(dst)[q] =
+                      make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+              } else {
+                for (int e = 0; e < 32 && key0 + e < p.Nk; ++e)
+                  dst[e] = uint16_t((e & 1) ? (dk[e >> 1] >> 16) : (dk[e >> 1] & 0xFFFFu));
+              }
+            }
+            tmem_st16(tmem + lane_base + L::kColG0 + hf * 32 + qt * 16, dk);
+          } else {
+            tmem_st16(tmem + lane_base + L::kColG0 + hf * 32 + qt * 16, pk);  // P^T
+            tmem_st16(tmem + lane_base + L::kColG1 + hf * 32 + qt * 16, dk);  // dS^T
+          }
         }
       }
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&bars[L::kBarGFull]);
-      if (t == 0) mbar_arrive(&bars[L::kBarStepEmpty + s]);  // bias tile read
+      if (t == 0) mbar_arrive(&bars[L::kBarStepEmpty + s]);  // this warpgroup's bias half read
     }
     // -------------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait<false>(&bars[L::kBarGDone], (nsteps - 1) & 1, wc);
-    ok = named_bar_and(1, kBwdTile, ok);  // every thread gets here; the loads below are warp-collective
+    // the warpgroup's threads all get here; the loads below are warp-collective
+    ok = named_bar_and(1 + g, kBwdTile, ok);
     if (ok) {
       tc_fence_after_sync();
       const int nrows = kB ? p.Nk : p.Nq;
-#pragma unroll 1
-      for (int a = 0; a < (kB ? 2 : 1); ++a) {
-        // A: dQ (acc0, scaled by tau).  B: a = 0 dK (acc0, scaled by tau), a = 1 dV (acc1)
+      {
+        // A: dQ (acc0, scaled by tau), columns 32g .. 32g+31 (D = 32: the
+        // first warpgroup alone).  B: warpgroup 0 dK (acc0, scaled by tau),
+        // warpgroup 1 dV (acc1), all D columns.
+        const int a = kB ? g : 0;
         const uint32_t col = (a == 0) ? L::kColAcc0 : L::kColAcc1;
         const float scale = (a == 0) ? p.tau : 1.f;
         float *dst = !kB ? p.dq : (a == 0 ? p.dk : p.dv);
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        const int c_begin = kB ? 0 : 32 * g, c_step = kB ? 32 : D;
+#pragma unroll 1
+        for (int c = c_begin; c < D; c += c_step) {
           uint32_t v[32];
           tmem_ld32(tmem + lane_base + col + c, v);
           tmem_wait_ld();
@@ -437,7 +465,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  if (warp == 5) tmem_dealloc(tmem, 512);
+  if (warp == kBwdWarpMma) tmem_dealloc(tmem, 512);
 }
 
 // Delta_i = sum_d dO_id O_id (bf16 inputs, fp32 sum), one warp per row.
