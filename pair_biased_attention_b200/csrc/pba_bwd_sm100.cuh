@@ -292,12 +292,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     for (int it = 0; it < nsteps && ok; ++it) {
       const int s = it % L::kStages;
       const int o0 = it * kBwdTile;
-      // S, dP and the step's tiles, and the previous step's accumulating MMAs
-      // (they read G0/G1, which this step overwrites).  The waits only set ok;
-      // the warpgroup leaves together at the barrier below.
+      // S, dP and the step's tiles.  The waits only set ok; the warpgroup
+      // leaves together at the barrier below.
       ok = mbar_wait<false>(&bars[L::kBarSFull], it & 1, wc);
       if (ok) ok = mbar_wait<false>(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
-      if (ok && it > 0) ok = mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc);
       const uint8_t *bt = smem + L::kOffBias + s * L::kBiasBytes;
       // Per-step column data in shared memory (double-buffered by step
       // parity); each warpgroup writes and reads only its own 64 columns, and
@@ -413,10 +411,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
                   reinterpret_cast<uint4 *>(dst)[q] =
                       make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
               } else {
-                for (int e = 0; e < 32 && key0 + e < p.Nk; ++e)
-                  dst[e] = uint16_t((e & 1) ? (dk[e >> 1] >> 16) : (dk[e >> 1] & 0xFFFFu));
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (key0 + e < p.Nk) dst[e] = uint16_t((e & 1) ? (dk[e >> 1] >> 16) : (dk[e >> 1] & 0xFFFFu));
               }
             }
+          }
+          if (qt == 0 && it > 0) {
+            // the previous step's accumulating MMAs read G0/G1, which the
+            // stores below overwrite: wait for them only now, so that they
+            // overlap this quarter's arithmetic
+            ok = mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc);
+            ok = named_bar_and(1 + g, kBwdTile, ok);
+            if (!ok) break;
+            tc_fence_after_sync();
+          }
+          if (!kB) {
             tmem_st16(tmem + lane_base + L::kColG0 + hf * 32 + qt * 16, dk);
           } else {
             tmem_st16(tmem + lane_base + L::kColG0 + hf * 32 + qt * 16, pk);  // P^T
@@ -424,6 +434,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
           }
         }
       }
+      if (!ok) break;
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&bars[L::kBarGFull]);
