@@ -288,10 +288,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     } else {
       key_ok = r < p.Nk && (mrow == nullptr || mrow[r] != 0);
     }
+    // Column data of a step, loaded from global memory one step ahead so
+    // that the loads' latency overlaps a step of work.  A: the mask bytes of
+    // this thread's key pair (threads t < 32); B: lse and Delta of this
+    // thread's query column (threads t < 64).
+    uint32_t nm0 = 1u, nm1 = 1u;
+    float nlse = 0.f, ndelta = 0.f;
+    auto load_cols = [&](int step) {
+      const int o = step * kBwdTile;
+      if (!kB) {
+        if (t < kBwdTile / 4 && mrow != nullptr) {
+          const int key = o + 2 * (g * (kBwdTile / 4) + t);
+          nm0 = key < p.Nk ? uint32_t(mrow[key]) : 0u;
+          nm1 = key + 1 < p.Nk ? uint32_t(mrow[key + 1]) : 0u;
+        }
+      } else if (t < kBwdTile / 2) {
+        const int qi = o + g * (kBwdTile / 2) + t;
+        if (qi < p.Nq) {
+          const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
+          nlse = p.lse[at];
+          ndelta = p.delta[at];
+        }
+      }
+    };
+    if (nsteps > 0) load_cols(0);
     bool ok = true;
     for (int it = 0; it < nsteps && ok; ++it) {
       const int s = it % L::kStages;
       const int o0 = it * kBwdTile;
+      const uint32_t cm0 = nm0, cm1 = nm1;
+      const float clse = nlse, cdelta = ndelta;
+      if (it + 1 < nsteps) load_cols(it + 1);
       // S, dP and the step's tiles.  The waits only set ok; the warpgroup
       // leaves together at the barrier below.
       ok = mbar_wait<false>(&bars[L::kBarSFull], it & 1, wc);
@@ -307,21 +334,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       if (!kB) {
         if (t < kBwdTile / 4) {
           const int pr = g * (kBwdTile / 4) + t;  // key pair of the step
-          uint32_t keep = 0;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int key = o0 + 2 * pr + e;
-            if (key < p.Nk && (mrow == nullptr || mrow[key] != 0)) keep |= 0xFFFFu << (16 * e);
-          }
+          const int key = o0 + 2 * pr;
+          const uint32_t keep = ((key < p.Nk && cm0 != 0u) ? 0x0000FFFFu : 0u) |
+                                ((key + 1 < p.Nk && cm1 != 0u) ? 0xFFFF0000u : 0u);
           reinterpret_cast<uint32_t *>(rv)[pr] = keep;
         }
       } else if (t < kBwdTile / 2) {
         const int col = g * (kBwdTile / 2) + t;  // query column of the step
         const int qi = o0 + col;
-        const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
-        const float lse = qi < p.Nq ? p.lse[at] : 0.f;
-        rv[col] = qi >= p.Nq ? -INFINITY : (lse == -INFINITY ? 0.f : -lse * l2e);  // see the A side
-        rv[kBwdTile + col] = qi < p.Nq ? -p.delta[at] : 0.f;
+        rv[col] = qi >= p.Nq ? -INFINITY : (clse == -INFINITY ? 0.f : -clse * l2e);  // see the A side
+        rv[kBwdTile + col] = qi < p.Nq ? -cdelta : 0.f;
       }
       ok = named_bar_and(1 + g, kBwdTile, ok);
       if (!ok) break;
