@@ -204,12 +204,14 @@ PBA_API pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, 
  *   o[s][i][h][:] = sum_j w[h][i][j] v[s][j][h][:]
  *   out = o * sigmoid(gate) (gate NULL: out = o);  lse[h][i] = natural log-sum-exp
  *   v, gate, out [S][N][H][D] bf16, device; bias [H][N][N] bf16, device;
- *   key_mask [N] uint8, device, or NULL; lse [H][N] float, device, or NULL.
+ *   key_mask [N] uint8, device, or NULL; lse [H][N] float, device (required:
+ *   the softmax is taken in two passes, lse first, then the weights
+ *   exp(bias - lse) times the values).
  * A row with no valid key gives out = 0 and lse = -inf.  D in {32, 64}
- * (else PBA_ERR_UNSUPPORTED); N a multiple of 8 and v, bias, gate, out
- * 16-byte aligned (else PBA_ERR_INVALID_ARG).  S = 0 or N = 0 writes nothing
- * and accepts NULL buffers.  The caller owns every buffer; nothing is
- * allocated.  Asynchronous on `stream`.
+ * (else PBA_ERR_UNSUPPORTED); N a multiple of 8, v, bias, gate, out 16-byte
+ * aligned and lse 4-byte aligned (else PBA_ERR_INVALID_ARG).  S = 0 or N = 0
+ * writes nothing and accepts NULL buffers.  The caller owns every buffer;
+ * nothing is allocated.  Asynchronous on `stream`.
  */
 PBA_API pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v, const void *bias,
                                const uint8_t *key_mask, const void *gate, void *out, float *lse, void *stream);

@@ -314,7 +314,9 @@ def tri_proj_forward(z, w_qkvg, w_b, H, out=None, bias=None, stream=None):
 
 def pwa_forward(v, bias, key_mask=None, gate=None, out=None, lse=None, return_lse=True, stream=None):
     """Pair weighted averaging, bf16: v, gate [S,N,H,D] (contiguous), bias
-    [H,N,N], key_mask [N] uint8 or None.  Returns out [S,N,H,D] and lse [H,N]."""
+    [H,N,N], key_mask [N] uint8 or None.  Returns out [S,N,H,D] and lse [H,N]
+    (the kernels always write lse; return_lse=False only drops it from the
+    result)."""
     for n, t in (("v", v), ("bias", bias), ("gate", gate)):
         _cuda(n, t, torch.bfloat16)
         if t is not None and not t.is_contiguous():
@@ -327,13 +329,12 @@ def pwa_forward(v, bias, key_mask=None, gate=None, out=None, lse=None, return_ls
         raise ValueError("key_mask must be a contiguous [N] uint8 tensor")
     if out is None:
         out = torch.empty_like(v)
-    if lse is None and return_lse:
-        lse = torch.empty((H, N), dtype=torch.float32, device=v.device)
+    lse_out = lse if lse is not None else torch.empty((H, N), dtype=torch.float32, device=v.device)
     _cuda("out", out, torch.bfloat16)
-    _cuda("lse", lse, torch.float32)
+    _cuda("lse", lse_out, torch.float32)
     _check("pwa_forward", load_library().pwa_forward(S, N, H, D, _ptr(v), _ptr(bias), _ptr(key_mask), _ptr(gate),
-                                                     _ptr(out), _ptr(lse), _stream(stream)))
-    return out, lse
+                                                     _ptr(out), _ptr(lse_out), _stream(stream)))
+    return out, (lse_out if (lse is not None or return_lse) else None)
 
 
 def pba_backward(q, k, v, bias, key_mask, out, lse, dout, softmax_scale=None, stream=None):

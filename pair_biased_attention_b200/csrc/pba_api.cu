@@ -393,10 +393,6 @@ cudaError_t launch_pwa(const pba::PwaParams &p, int grid, cudaStream_t stream) {
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
     attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
-    cudaFuncAttributes fa;
-    if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
-        fa.numRegs * pba::kPwaThreads < pba::kPwaRegSplitTotal)
-      attr_err = cudaErrorInvalidConfiguration;
   });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kPwaThreads, L::kSmemAlloc, stream>>>(p);
@@ -603,12 +599,13 @@ pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v
   if (D != 32 && D != 64) return PBA_ERR_UNSUPPORTED;
   if (N % 8 != 0) return PBA_ERR_INVALID_ARG;  // bias rows are tile rows: 16-byte strides
   if (S == 0 || N == 0) return PBA_OK;        // nothing to write; zero-extent buffers may be NULL
-  if (v == nullptr || bias == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
-  if (!aligned16(v) || !aligned16(bias) || !aligned16(out) || (gate != nullptr && !aligned16(gate)))
+  if (v == nullptr || bias == nullptr || out == nullptr || lse == nullptr) return PBA_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(bias) || !aligned16(out) || (gate != nullptr && !aligned16(gate)) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return PBA_ERR_INVALID_ARG;
   pba_status s = check_device();
   if (s != PBA_OK) return s;
-  const int slabs = 192 / int(D);
+  const int slabs = pba::kPwaDF / int(D);
   pba::PwaParams p;
   std::memset(&p, 0, sizeof(p));
   {
@@ -629,7 +626,7 @@ pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v
   p.S = int(S);
   p.N = int(N);
   p.H = int(H);
-  p.n_qblocks = int((N + pba::kPwaQTiles * pba::kPwaBM - 1) / (pba::kPwaQTiles * pba::kPwaBM));
+  p.n_qblocks = int((N + pba::kPwaBM - 1) / pba::kPwaBM);
   p.n_ftiles = int((S + slabs - 1) / slabs);
   const int64_t n_units = int64_t(H) * p.n_qblocks * p.n_ftiles;
   if (n_units > kMaxI32) return PBA_ERR_INVALID_ARG;
@@ -649,6 +646,13 @@ pba_status pwa_forward(int64_t S, int64_t N, int64_t H, int64_t D, const void *v
     return PBA_ERR_CUDA;
   const int grid = int(std::min<int64_t>(n_units, sms));
   cudaStream_t st = static_cast<cudaStream_t>(stream_ptr);
+  // first pass: the log-sum-exp of every weight row (one warp per row)
+  const int64_t rows = H * N;
+  const int mask_vec8 = key_mask != nullptr && (reinterpret_cast<uintptr_t>(key_mask) & 7u) == 0;
+  pba::pba_pwa_lse_kernel<<<int((rows * 32 + 255) / 256), 256, 0, st>>>(static_cast<const uint16_t *>(bias), key_mask,
+                                                                         mask_vec8, lse, int(N), rows);
+  if (cudaGetLastError() != cudaSuccess) return PBA_ERR_CUDA;
+  // second pass: the normalised weights times the values
   cudaError_t e = (D == 64) ? dispatch_pwa<64>(p, grid, gate != nullptr, st)
                             : dispatch_pwa<32>(p, grid, gate != nullptr, st);
   return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;

@@ -178,7 +178,11 @@ def test_pwa_rejects_null_and_unaligned(lib):
     assert lib.pwa_forward(4, 64, 2, 32, None, FAKE, None, None, FAKE, None, None) == pba.PBA_ERR_INVALID_ARG
     assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, None, None, None, None) == pba.PBA_ERR_INVALID_ARG
     odd = ctypes.c_void_p(0x10008)
-    assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, odd, FAKE, None, None) == pba.PBA_ERR_INVALID_ARG
+    assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, odd, FAKE, FAKE, None) == pba.PBA_ERR_INVALID_ARG
+    # lse is required: the softmax takes it as its first pass
+    assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, None, FAKE, None, None) == pba.PBA_ERR_INVALID_ARG
+    assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, None, FAKE, ctypes.c_void_p(0x10002),
+                           None) == pba.PBA_ERR_INVALID_ARG
 
 
 def test_selftest_rejects_bad_limit(lib):
