@@ -63,6 +63,13 @@ constexpr uint32_t kPwaColO = 0;
 constexpr uint32_t kPwaColP = kPwaDF;  // P0; P1 follows after kPwaBN / 2 columns
 static_assert(kPwaColP + 2 * (kPwaBN / 2) <= kPwaTmemCols, "Tensor Memory budget");
 static_assert(kPwaGroupKeys == 32, "one 16-column Tensor Memory store per warpgroup and tile");
+// One key pair in PBA_PWA_EXP_EMU_EVERY takes the software exp2 on the FMA
+// pipe (0: none).  With sixteen softmax warps the exp2 unit is not the limit
+// here (measured at S=64, N=4096, H=8, D=32: every third pair 0.72 ms, none
+// 0.70 ms), so all pairs use the unit.
+#ifndef PBA_PWA_EXP_EMU_EVERY
+#define PBA_PWA_EXP_EMU_EVERY 0
+#endif
 
 struct PwaParams {
   CUtensorMap tm_v;     // v [S][N][H][D] as (D, N, H, S), box {D, 128, 1, kSlabs}
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(256) pba_pwa_lse_kernel(const uint16_t *bias, 
 template <int D, bool kGate, bool kMasked>
 __global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __grid_constant__ PwaParams p) {
   using L = PwaLayout<D>;
-  constexpr int kExpEmuEvery = (D == 32) ? PBA_EXP_EMU_EVERY_D32 : PBA_EXP_EMU_EVERY_D64;
+  constexpr int kExpEmuEvery = PBA_PWA_EXP_EMU_EVERY;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
@@ -368,13 +375,21 @@ __global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __g
     const int box = (g * kPwaGroupKeys) / 64, chunk0 = ((g * kPwaGroupKeys) % 64) / 8;
     bool ok = true;
     int gt = 0, uc = 0;
+    // the row's lse, loaded one unit ahead
+    auto load_lse = [&](int uu) -> float {
+      if (uu >= p.n_units) return -INFINITY;
+      const PwaUnit nu = decode_pwa_unit(p, uu);
+      return nu.q0 + t < p.N ? p.lse[int64_t(nu.h) * p.N + nu.q0 + t] : -INFINITY;
+    };
+    float next_lse = load_lse(u_begin);
     for (int u = u_begin; u < p.n_units && ok; u += u_step, ++uc) {
       const PwaUnit un = decode_pwa_unit(p, u);
       const int row = un.q0 + t;
       const bool live = row < p.N;
       // -lse*log2(e) of the row; a row with no valid key has lse = -inf and
       // -inf logits only, which the finite stand-in 0 keeps at weight 0
-      const float lse_r = live ? p.lse[int64_t(un.h) * p.N + row] : -INFINITY;
+      const float lse_r = next_lse;
+      next_lse = load_lse(u + u_step);
       const float neg = (lse_r == -INFINITY) ? 0.f : -lse_r * kLog2e;
       const float2 neg2 = make_float2(neg, neg);
       for (int j = 0; j < nt; ++j, ++gt) {
