@@ -417,9 +417,11 @@ def run_proj(args, pba, tcfg, dev, stream, pg, peaks):
 def run_pwa(args, pba, dev, stream, pg, peaks, clk):
     """Pair weighted averaging on pwa4k (S=64 sequences, N=4096, H=8, D=32,
     gate, 5% key padding), timed on its own after the step: K calls after 3
-    warm-up calls, CUDA events on the stream.  Compute-bound: 2*H*S*N^2*D
-    FLOPs on the tensor cores and H*N^2 exps per 192-feature tile on the
-    exp2 unit (16 per clock per SM)."""
+    warm-up calls, CUDA events on the stream; a call is the row log-sum-exp
+    pass and the weights-times-values kernel (2 launches).  Compute-bound:
+    2*H*S*N^2*D FLOPs on the tensor cores; H*N^2 exps in the first pass and
+    H*N^2 per 256-feature tile in the second on the exp2 unit (16 per clock
+    per SM)."""
     cfg = W.PWA4K
     v, bias, mask, gate = W.pwa_inputs(cfg, dev)
     out = torch.empty_like(v)
@@ -438,12 +440,12 @@ def run_pwa(args, pba, dev, stream, pg, peaks, clk):
         raise RuntimeError("the pair weighted averaging kernel recorded a device error")
     ms = max_over_ranks(s.elapsed_time(e), pg) / args.steps
     flops = 2.0 * cfg.H * cfg.S * cfg.N * cfg.N * cfg.D
-    ftiles = -(-cfg.S // (192 // cfg.D))
-    exps = cfg.H * cfg.N * cfg.N * ftiles
+    ftiles = -(-cfg.S // (256 // cfg.D))
+    exps = cfg.H * cfg.N * cfg.N * (ftiles + 1)
     tflops = flops / (ms / 1e3) / 1e12
     sm_hz = (clk.get("sm_mhz") or 1965.0) * 1e6 if isinstance(clk, dict) else 1965e6
     exp_floor_ms = exps / (16 * torch.cuda.get_device_properties(dev).multi_processor_count * sm_hz) * 1e3
-    return {"ms_per_call": ms, "calls": args.steps, "gpu_launches": args.steps, "tflops": tflops,
+    return {"ms_per_call": ms, "calls": args.steps, "gpu_launches": 2 * args.steps, "tflops": tflops,
             "workload": f"pwa4k: S={cfg.S} N={cfg.N} H={cfg.H} D={cfg.D}, gate, 5% key padding, bias [H,N,N]",
             "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": tflops / peaks["bf16_tflops"], "kernel": "pba_pwa_sm100_kernel (pwa_forward)",
