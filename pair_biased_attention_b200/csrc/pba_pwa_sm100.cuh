@@ -133,59 +133,94 @@ __device__ __forceinline__ PwaUnit decode_pwa_unit(const PwaParams &p, int u) {
 
 // lse[row] = natural log of the sum over valid keys j of exp(bias[row][j]);
 // -inf for a row with no valid key.  One warp per row of N (a multiple of 8)
-// bf16 logits, each lane an online maximum and sum over 8-key chunks, merged
-// across the warp at the end.
+// bf16 logits.  Each lane keeps an online maximum and a sum over 16-key
+// steps (two 8-key chunks 32 chunks apart, so the warp's loads stay
+// coalesced): masked keys become bf16 -inf through keep words, the step's
+// maximum is taken once, and the exponents and sums run two keys per packed
+// operation.  The lanes are merged at the end.
 __global__ void __launch_bounds__(256) pba_pwa_lse_kernel(const uint16_t *bias, const uint8_t *mask, int mask_vec8,
                                                           float *lse, int N, int64_t rows) {
   const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;  // the same for every lane of the warp
   const uint4 *src = reinterpret_cast<const uint4 *>(bias + row * int64_t(N));
-  float m = -INFINITY, s = 0.f;
-#pragma unroll 4
-  for (int c = lane; c < N / 8; c += 32) {
-    const uint4 w4 = __ldg(src + c);
-    const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-    float xs[8];
+  const int nch = N / 8;  // 8-key chunks
+  const float2 l2e2 = make_float2(kLog2e, kLog2e);
+  float m = -INFINITY;
+  float2 s2 = make_float2(0.f, 0.f);
+  // keep words of the 8 keys from 8 mask bytes: 0xFFFF per key that takes part
+  auto keep8 = [&](int c, uint32_t (&k)[4]) {
+    uint32_t mb0, mb1;
+    if (mask_vec8) {
+      const uint2 m2 = __ldg(reinterpret_cast<const uint2 *>(mask + 8 * c));
+      mb0 = m2.x;
+      mb1 = m2.y;
+    } else {
+      mb0 = mb1 = 0u;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      xs[2 * e] = bf16lo_to_f32(wv[e]);
-      xs[2 * e + 1] = bf16hi_to_f32(wv[e]);
+      for (int q = 0; q < 4; ++q) {
+        mb0 |= uint32_t(__ldg(mask + 8 * c + q)) << (8 * q);
+        mb1 |= uint32_t(__ldg(mask + 8 * c + 4 + q)) << (8 * q);
+      }
+    }
+    const uint32_t v0 = __vcmpne4(mb0, 0u), v1 = __vcmpne4(mb1, 0u);  // 0xFF per byte that is nonzero
+    k[0] = __byte_perm(v0, 0u, 0x1100);
+    k[1] = __byte_perm(v0, 0u, 0x3322);
+    k[2] = __byte_perm(v1, 0u, 0x1100);
+    k[3] = __byte_perm(v1, 0u, 0x3322);
+  };
+  for (int c = lane; c < nch; c += 64) {
+    uint32_t w[8];
+    const bool second = c + 32 < nch;
+    {
+      const uint4 a = __ldg(src + c);
+      const uint4 b = second ? __ldg(src + c + 32) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
     }
     if (mask != nullptr) {
-      uint32_t mb[2];
-      if (mask_vec8) {
-        const uint2 m2 = __ldg(reinterpret_cast<const uint2 *>(mask + 8 * c));
-        mb[0] = m2.x;
-        mb[1] = m2.y;
+      uint32_t k[8];
+      keep8(c, *reinterpret_cast<uint32_t(*)[4]>(&k[0]));
+      if (second) {
+        keep8(c + 32, *reinterpret_cast<uint32_t(*)[4]>(&k[4]));
       } else {
-        mb[0] = mb[1] = 0u;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mb[k >> 2] |= uint32_t(__ldg(mask + 8 * c + k)) << (8 * (k & 3));
+        for (int e = 4; e < 8; ++e) k[e] = 0xFFFFFFFFu;  // already -inf
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (((mb[k >> 2] >> (8 * (k & 3))) & 0xFFu) == 0u) xs[k] = -INFINITY;
+      for (int e = 0; e < 8; ++e) w[e] = (w[e] & k[e]) | (~k[e] & 0xFF80FF80u);
     }
-    float cm = xs[0];
+    float2 x[8];
 #pragma unroll
-    for (int k = 1; k < 8; ++k) cm = fmaxf(cm, xs[k]);
+    for (int e = 0; e < 8; ++e) x[e] = make_float2(bf16lo_to_f32(w[e]), bf16hi_to_f32(w[e]));
+    float cm = fmaxf(x[0].x, x[0].y);
+#pragma unroll
+    for (int e = 1; e < 8; ++e) cm = max3f(cm, x[e].x, x[e].y);
     if (cm > m) {
-      s = (m == -INFINITY) ? 0.f : s * ex2_approx((m - cm) * kLog2e);
+      if (m != -INFINITY) {
+        const float a = ex2_approx((m - cm) * kLog2e);
+        s2 = fmul2(s2, make_float2(a, a));
+      }
       m = cm;
     }
     if (m != -INFINITY) {
+      const float neg = -m * kLog2e;
+      const float2 neg2 = make_float2(neg, neg);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) s += ex2_approx((xs[k] - m) * kLog2e);
+      for (int e = 0; e < 8; ++e) {
+        const float2 a = ffma2(x[e], l2e2, neg2);
+        s2 = fadd2(s2, make_float2(ex2_approx(a.x), ex2_approx(a.y)));
+      }
     }
   }
+  float s = s2.x + s2.y;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float t2 = __shfl_xor_sync(0xffffffffu, s, o);
     const float mm = fmaxf(m, m2);
     s = ((m == -INFINITY) ? 0.f : s * ex2_approx((m - mm) * kLog2e)) +
-        ((m2 == -INFINITY) ? 0.f : s2 * ex2_approx((m2 - mm) * kLog2e));
+        ((m2 == -INFINITY) ? 0.f : t2 * ex2_approx((m2 - mm) * kLog2e));
     m = mm;
   }
   if (lane == 0) lse[row] = (m == -INFINITY) ? -INFINITY : m + logf(s);
