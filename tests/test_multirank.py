@@ -13,7 +13,10 @@ import bench
 
 
 def _init(rank, world, rendezvous):
-    # a file rendezvous: no TCP port to collide with other processes
+    # a file rendezvous: no TCP port to collide with other processes; the
+    # ranks' own gloo sockets on the loopback interface, whatever the host
+    # name resolves to
+    os.environ.setdefault("GLOO_SOCKET_IFNAME", "lo")
     dist.init_process_group("gloo", init_method=f"file://{rendezvous}", rank=rank, world_size=world)
 
 
