@@ -51,7 +51,10 @@ constexpr int kPwaBN = 128;                          // keys per tile
 constexpr int kPwaGroups = 4;                        // softmax warpgroups
 constexpr int kPwaGroupKeys = kPwaBN / kPwaGroups;   // keys of a tile per warpgroup
 constexpr int kPwaDF = 256;                          // features per unit
-constexpr int kPwaBiasStages = 2;
+#ifndef PBA_PWA_BIAS_STAGES
+#define PBA_PWA_BIAS_STAGES 2
+#endif
+constexpr int kPwaBiasStages = PBA_PWA_BIAS_STAGES;  // bias tiles in flight
 constexpr int kPwaSoftmaxWarps = 4 * kPwaGroups;
 constexpr int kPwaThreads = 32 * (kPwaSoftmaxWarps + 4);
 constexpr int kPwaWarpProducer = kPwaSoftmaxWarps;

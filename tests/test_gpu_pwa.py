@@ -61,12 +61,13 @@ def test_pwa512_full(cuda_device):
 
 
 @pytest.mark.parametrize("S,N,H,D,mask_frac,gate", [
-    (6, 256, 2, 32, 0.0, False),    # one feature tile exactly, whole key tiles, no mask
-    (7, 200, 3, 32, 0.1, True),     # ragged last feature tile and key tile
-    (2, 128, 4, 32, 0.0, True),     # fewer sequences than a feature tile
-    (5, 384, 2, 64, 0.2, True),     # D = 64 (3 sequences per feature tile)
+    (8, 256, 2, 32, 0.0, False),    # one 256-feature tile exactly, whole key tiles, no mask
+    (6, 256, 2, 32, 0.0, False),    # fewer sequences than a feature tile
+    (7, 200, 3, 32, 0.1, True),     # ragged key tile, ragged row block
+    (2, 128, 4, 32, 0.0, True),     # one key tile, one row block
+    (5, 384, 2, 64, 0.2, True),     # D = 64 (4 sequences per feature tile): a ragged second tile
     (3, 1000, 1, 64, 0.5, False),   # long rows, half the keys masked
-    (13, 520, 2, 32, 0.05, True),   # several units per CTA
+    (13, 520, 2, 32, 0.05, True),   # several units per CTA, ragged second feature tile
 ])
 def test_shapes(cuda_device, S, N, H, D, mask_frac, gate):
     _run(f"pwa S={S} N={N} H={H} D={D}", *_rand(S, N, H, D, seed=S * 31 + N, device=cuda_device,
@@ -92,6 +93,16 @@ def test_uniform_logits_give_mean_of_values(cuda_device):
     mean = v.float()[:, mask.bool()].mean(dim=1, keepdim=True)
     assert (out.float() - mean).abs().max().item() <= 1e-2
     assert torch.allclose(lse, torch.full_like(lse, math.log(int(mask.sum()))), atol=1e-4)
+
+
+def test_unaligned_key_mask(cuda_device):
+    """A key mask at an odd address: both passes read it byte by byte."""
+    v, bias, mask, gate = _rand(9, 264, 2, 32, seed=21, device=cuda_device, mask_frac=0.25)
+    buf = torch.zeros((mask.numel() + 1,), dtype=torch.uint8, device=cuda_device)
+    buf[1:] = mask
+    odd = buf[1:]
+    assert odd.data_ptr() % 8 != 0
+    _run("pwa unaligned mask", v, bias, odd, gate)
 
 
 def test_zero_sizes(cuda_device):
