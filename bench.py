@@ -364,6 +364,7 @@ def main():
     }
 
     line["tri_proj"] = run_proj(args, pba, tcfg, dev, stream, pg, peaks)
+    line["tri_out_proj"] = run_out_proj(args, pba, tcfg, dev, stream, pg, peaks)
     line["pwa"] = run_pwa(args, pba, dev, stream, pg, peaks, clk)
     line["backward"] = run_bwd(args, pba, dev, stream, pg, peaks)
     if not args.no_e2e:
@@ -411,6 +412,41 @@ def run_proj(args, pba, tcfg, dev, stream, pg, peaks):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
                          "kernel": "pba_proj_sm100_kernel (tri_proj_forward)", "peak_source": peaks["source"],
+                         "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
+
+
+def run_out_proj(args, pba, tcfg, dev, stream, pg, peaks):
+    """The output projection of the triangle workload (tri_out_proj_forward:
+    o [N,N,H,D] -> out [N,N,c] = o W_o), timed on its own after the step: K
+    calls after 3 warm-up calls, CUDA events on the stream.  HBM-bound:
+    algorithmic bytes = o read once + out written once (+ W_o)."""
+    g = torch.Generator(dev.type).manual_seed(tcfg.seed + 100)
+    HD = tcfg.H * tcfg.D
+    o = torch.randn((tcfg.N, tcfg.N, tcfg.H, tcfg.D), generator=g, device=dev).to(torch.bfloat16)
+    w_o = (torch.randn((HD, tcfg.c), generator=g, device=dev) / HD ** 0.5).to(torch.bfloat16)
+    out = torch.empty((tcfg.N, tcfg.N, tcfg.c), dtype=torch.bfloat16, device=dev)
+    call = lambda: pba.tri_out_proj_forward(o, w_o, out=out, stream=stream)
+    for _ in range(3):
+        call()
+    barrier(pg)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(args.steps):
+        call()
+    e.record(stream)
+    barrier(pg)
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("the output projection kernel recorded a device error")
+    ms = max_over_ranks(s.elapsed_time(e), pg) / args.steps
+    N2 = tcfg.N * tcfg.N
+    nbytes = N2 * HD * 2 + N2 * tcfg.c * 2 + HD * tcfg.c * 2
+    flops = 2.0 * N2 * HD * tcfg.c
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"ms_per_call": ms, "calls": args.steps, "gpu_launches": args.steps,
+            "workload": f"tri{tcfg.N}: o [{tcfg.N},{tcfg.N},{tcfg.H},{tcfg.D}] bf16 -> out [N,N,{tcfg.c}]",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
+                         "kernel": "pba_oproj_sm100_kernel (tri_out_proj_forward)", "peak_source": peaks["source"],
                          "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
 
 

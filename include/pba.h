@@ -195,6 +195,25 @@ PBA_API pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, 
                                     const void *w_b, void *q, void *k, void *v, void *g, void *bias, void *stream);
 
 /*
+ * tri_out_proj_forward -- the output projection of triangle attention back
+ * to the pair channels (Fold-CP, Figure 2(a): triangle attention reads the
+ * pair representation and its result returns to it; the pages fix no layout
+ * for this map, and a plain linear map of the concatenated heads is the
+ * reading taken here):
+ *   o     [N][N][H][D] bf16, device (tri_attn_forward's output; H*D = 128)
+ *   w_o   [H*D][c]     bf16, device
+ *   out   [N][N][c]    bf16, device
+ * out[r][:] = o[r][:] W_o for every pair row r = i*N + j, in fp32 sums of the
+ * bf16 products, rounded once to bf16.  Requires H*D = 128 and c in {64, 128}
+ * (else PBA_ERR_UNSUPPORTED), N <= 32768 and o, w_o, out 16-byte aligned
+ * (else PBA_ERR_INVALID_ARG).  N = 0 does nothing and accepts NULL buffers.
+ * The caller owns every buffer; nothing is allocated.  Asynchronous on
+ * `stream`.
+ */
+PBA_API pba_status tri_out_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const void *o, const void *w_o,
+                                        void *out, void *stream);
+
+/*
  * pwa_forward -- pair weighted averaging (Fold-CP, Table 1 row "Pair
  * Weighted Avg.", serial time B*H*S*N^2*D, distributed as a "2D ring + tiled
  * softmax"; Figure 2 groups it with the ring attention, a softmax whose

@@ -229,6 +229,18 @@ def tri_proj(z, w, wb, rows=None, nthreads: int = 0, mutant: int = 0):
     return {"out": out, "bias": bias}
 
 
+def tri_out_proj(o, w_o, rows=None, nthreads: int = 0, mutant: int = 0):
+    """Output projection of triangle attention in fp64: o [N,N,H,D] (or
+    [R, H*D]), w_o [H*D, c]; out[r] = o[r] (heads concatenated, h major) W_o.
+    The same linear map as the input projections, so it runs through
+    oracle_tri_proj with no bias columns.  Returns out [R, c] for the selected
+    flat pair rows (None = all)."""
+    of = _f64(o)
+    of = of.reshape(-1, of.shape[-2] * of.shape[-1]) if of.ndim == 4 else of.reshape(-1, of.shape[-1])
+    r = tri_proj(of, w_o, np.zeros((of.shape[1], 1)), rows=rows, nthreads=nthreads, mutant=mutant)
+    return r["out"]
+
+
 def pwa(v, bias, key_mask=None, g=None, nthreads: int = 0, mutant: int = 0):
     """Pair weighted averaging in fp64 (the reading stated in pba_oracle.c):
     v [S,N,H,D], bias [H,N,N], key_mask [N] or None, g [S,N,H,D] or None.

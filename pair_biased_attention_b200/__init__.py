@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "PbaError", "PBA_OK", "PBA_ERR_INVALID_ARG", "PBA_ERR_UNSUPPORTED", "PBA_ERR_CUDA", "PBA_ERR_TIMEOUT",
-    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pwa_forward", "pba_backward",
+    "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "tri_out_proj_forward", "pwa_forward", "pba_backward",
     "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_selftest_exp2",
     "pba_status_string",
 ]
@@ -83,6 +83,8 @@ def load_library() -> ctypes.CDLL:
     lib.tri_attn_forward.restype = st
     lib.tri_proj_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 9
     lib.tri_proj_forward.restype = st
+    lib.tri_out_proj_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 4
+    lib.tri_out_proj_forward.restype = st
     lib.pwa_forward.argtypes = [ctypes.c_int64] * 4 + [_p] * 7
     lib.pwa_forward.restype = st
     lib.pba_backward.argtypes = [desc_p] + [_p] * 14
@@ -310,6 +312,27 @@ def tri_proj_forward(z, w_qkvg, w_b, H, out=None, bias=None, stream=None):
                                                                _ptr(k), _ptr(v), _ptr(g), _ptr(bias),
                                                                _stream(stream)))
     return q, k, v, g, bias
+
+
+def tri_out_proj_forward(o, w_o, out=None, stream=None):
+    """Output projection of triangle attention, bf16: o [N,N,H,D]
+    (contiguous, H*D = 128), w_o [H*D, c].  Returns out [N,N,c] = o W_o."""
+    for n, t in (("o", o), ("w_o", w_o)):
+        _cuda(n, t, torch.bfloat16)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    N, N2, H, D = o.shape
+    if N2 != N or w_o.dim() != 2 or w_o.shape[0] != H * D:
+        raise ValueError("o must be [N,N,H,D] and w_o [H*D, c]")
+    c = w_o.shape[1]
+    if out is None:
+        out = torch.empty((N, N, c), dtype=torch.bfloat16, device=o.device)
+    _cuda("out", out, torch.bfloat16)
+    if not out.is_contiguous() or tuple(out.shape) != (N, N, c):
+        raise ValueError("out must be a contiguous [N,N,c] tensor")
+    _check("tri_out_proj_forward", load_library().tri_out_proj_forward(N, c, H, D, _ptr(o), _ptr(w_o), _ptr(out),
+                                                                       _stream(stream)))
+    return out
 
 
 def pwa_forward(v, bias, key_mask=None, gate=None, out=None, lse=None, return_lse=True, stream=None):

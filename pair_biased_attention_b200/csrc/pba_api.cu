@@ -15,6 +15,7 @@
 #include "pba.h"
 #include "pba_attn_sm100.cuh"
 #include "pba_proj_sm100.cuh"
+#include "pba_oproj_sm100.cuh"
 #include "pba_pwa_sm100.cuh"
 #include "pba_bwd_sm100.cuh"
 #include "pba_simt.cuh"
@@ -384,6 +385,20 @@ cudaError_t launch_proj(const pba::ProjParams &p, int grid, cudaStream_t stream)
   return cudaGetLastError();
 }
 
+template <int kC>
+cudaError_t launch_oproj(const pba::OprojParams &p, int grid, cudaStream_t stream) {
+  using L = pba::OprojLayout<kC>;
+  auto kern = pba::pba_oproj_sm100_kernel<kC>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, pba::kOprojThreads, L::kSmemAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------ pair weighted averaging
 template <int D, bool kGate, bool kMasked>
 cudaError_t launch_pwa(const pba::PwaParams &p, int grid, cudaStream_t stream) {
@@ -590,6 +605,52 @@ pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const vo
                   : H == 2 ? launch_proj<2>(p, grid, st)
                   : H == 4 ? launch_proj<4>(p, grid, st)
                            : launch_proj<8>(p, grid, st);
+  return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
+pba_status tri_out_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const void *o, const void *w_o,
+                                void *out, void *stream_ptr) {
+  if (N < 0 || N > 32768 || H < 1 || D < 1) return PBA_ERR_INVALID_ARG;
+  if ((c != 64 && c != 128) || H * D != pba::kOprojK) return PBA_ERR_UNSUPPORTED;
+  if (N == 0) return PBA_OK;  // nothing to read or write; zero-extent buffers may be NULL
+  if (o == nullptr || w_o == nullptr || out == nullptr) return PBA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(out)) return PBA_ERR_INVALID_ARG;
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  const int64_t rows = N * N;
+  pba::OprojParams p;
+  std::memset(&p, 0, sizeof(p));
+  {
+    const uint64_t dims[4] = {uint64_t(pba::kOprojK), uint64_t(rows), 1, 1};
+    const int64_t st[3] = {int64_t(pba::kOprojK) * 2, 0, 0};
+    const uint32_t box[4] = {64, uint32_t(pba::kOprojRows), 1, 1};
+    if (!make_map(&p.tm_o, o, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+  }
+  {
+    // W_o [128][c]: 64-column slabs of all 128 rows
+    const uint64_t dims[4] = {uint64_t(c), uint64_t(pba::kOprojK), 1, 1};
+    const int64_t st[3] = {c * 2, 0, 0};
+    const uint32_t box[4] = {64, uint32_t(pba::kOprojK), 1, 1};
+    if (!make_map(&p.tm_w, w_o, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+  }
+  {
+    const uint64_t dims[4] = {uint64_t(c), uint64_t(rows), 1, 1};
+    const int64_t st[3] = {c * 2, 0, 0};
+    const uint32_t box[4] = {32, uint32_t(pba::kOprojRows), 1, 1};
+    if (!make_map(&p.tm_out, out, dims, st, box, CU_TENSOR_MAP_SWIZZLE_64B)) return PBA_ERR_INVALID_ARG;
+  }
+  p.rows = rows;
+  p.n_tiles = int((rows + pba::kOprojRows - 1) / pba::kOprojRows);
+  p.err = device_error_word();
+  if (p.err == nullptr) return PBA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return PBA_ERR_CUDA;
+  const int grid = std::min(p.n_tiles, sms);
+  cudaStream_t st = static_cast<cudaStream_t>(stream_ptr);
+  const cudaError_t e = c == 64 ? launch_oproj<64>(p, grid, st) : launch_oproj<128>(p, grid, st);
   return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
 }
 

@@ -28,7 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "pwa_forward",
+    for n in ("pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward",
+              "tri_out_proj_forward", "pwa_forward",
               "pba_status_string",
               "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout",
               "pba_selftest_exp2"):
@@ -183,6 +184,26 @@ def test_pwa_rejects_null_and_unaligned(lib):
     assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, None, FAKE, None, None) == pba.PBA_ERR_INVALID_ARG
     assert lib.pwa_forward(4, 64, 2, 32, FAKE, FAKE, None, None, FAKE, ctypes.c_void_p(0x10002),
                            None) == pba.PBA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("N,c,H,D,expect", [
+    (16, 96, 4, 32, pba.PBA_ERR_UNSUPPORTED),   # pair channels
+    (16, 128, 4, 16, pba.PBA_ERR_UNSUPPORTED),  # H*D != 128
+    (-1, 128, 4, 32, pba.PBA_ERR_INVALID_ARG),
+    (40000, 128, 4, 32, pba.PBA_ERR_INVALID_ARG),
+])
+def test_out_proj_rejects_bad_shapes(lib, N, c, H, D, expect):
+    assert lib.tri_out_proj_forward(N, c, H, D, FAKE, FAKE, FAKE, None) == expect
+
+
+def test_out_proj_rejects_null_and_unaligned(lib):
+    assert lib.tri_out_proj_forward(0, 128, 4, 32, None, None, None, None) == pba.PBA_OK  # nothing to do
+    for i in range(3):
+        args = [FAKE, FAKE, FAKE]
+        args[i] = None
+        assert lib.tri_out_proj_forward(16, 128, 4, 32, *args, None) == pba.PBA_ERR_INVALID_ARG
+        args[i] = ctypes.c_void_p(0x10008)
+        assert lib.tri_out_proj_forward(16, 128, 4, 32, *args, None) == pba.PBA_ERR_INVALID_ARG
 
 
 def test_selftest_rejects_bad_limit(lib):

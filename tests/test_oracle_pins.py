@@ -396,6 +396,30 @@ def test_proj_linearity_and_row_selection():
     assert np.array_equal(rs["out"], r1["out"][rows]) and np.array_equal(rs["bias"], r1["bias"][:, rows])
 
 
+# The output projection maps the concatenated heads of triangle attention back
+# to the pair channels: out[r] = o[r, h*D + d] W_o.  Pinned on the flattening
+# of (h, d), which is where a plausible mistake would sit.
+def test_out_proj_one_hot_head_and_dim_select_weight_row():
+    rng = np.random.default_rng(3)
+    H, D, c = 4, 8, 16
+    w_o = rng.standard_normal((H * D, c))
+    o = np.zeros((2, 2, H, D))
+    o[0, 1, 2, 5] = 1.0  # pair row 1 (i = 0, j = 1): head 2, dim 5 -> weight row 2*8 + 5
+    o[1, 0, 0, 7] = -2.0  # pair row 2: head 0, dim 7 -> -2 x weight row 7
+    out = oracle.tri_out_proj(o, w_o)
+    assert out.shape == (4, c)
+    assert np.array_equal(out[1], w_o[21]) and np.array_equal(out[2], -2.0 * w_o[7])
+    assert not out[0].any() and not out[3].any()
+
+
+def test_out_proj_identity_and_numpy():
+    rng = np.random.default_rng(4)
+    o = rng.standard_normal((3, 3, 2, 4))
+    assert np.array_equal(oracle.tri_out_proj(o, np.eye(8)), o.reshape(9, 8))
+    w = rng.standard_normal((8, 5))
+    assert np.abs(oracle.tri_out_proj(o, w) - o.reshape(9, 8) @ w).max() < 1e-12
+
+
 # ---------------------------------------------------------------- pair weighted averaging
 # Fold-CP, Table 1 row "Pair Weighted Avg." (B*H*S*N^2*D; "2D ring + tiled
 # softmax") and Figure 2 (grouped with the ring attention's merged softmax).  Reading: a
