@@ -272,7 +272,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "pwa4k", "bwd4k"], default="none",
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "oproj1024", "pwa4k", "bwd4k"],
+                    default="none",
                     help="run one small case only (for ncu captures); prints no JSON line")
     args = ap.parse_args()
     world, rank, local, pg = dist_setup(args)
@@ -565,9 +566,11 @@ def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, fl
 
 
 def run_profile_case(args, pba, dev):
-    """One small case for ncu: pba4k = pba_forward at N=4096 (bias 512 MB,
-    larger than L2) after one warm-up launch; tri512 = triangle attention
-    N=512 both orientations."""
+    """One small case for ncu, each kernel launched twice (a warm-up launch,
+    then the captured one): pba4k = pba_forward at N=4096 (bias 512 MB, larger
+    than L2); tri512 = triangle attention N=512 both orientations; proj1024 /
+    oproj1024 = the input / output projections at tri1024; pwa4k = pwa_forward;
+    bwd4k = pba_backward at N=4096, H=4."""
     if args.profile == "bwd4k":
         q, k, v, bias, mask = W.random_attn(1, 4, 4096, 4096, 64, seed=12, device=dev, mask_frac=0.05)
         out, lse = pba.pba_forward(q, k, v, bias, mask)
@@ -582,6 +585,13 @@ def run_profile_case(args, pba, dev):
         z, w, wb = W.tri_pair_inputs(W.TRI1024, dev)
         for _ in range(2):
             pba.tri_proj_forward(z, w, wb, W.TRI1024.H)
+    elif args.profile == "oproj1024":
+        cfg = W.TRI1024
+        g = torch.Generator(dev.type).manual_seed(cfg.seed + 100)
+        o = torch.randn((cfg.N, cfg.N, cfg.H, cfg.D), generator=g, device=dev).to(torch.bfloat16)
+        w_o = (torch.randn((cfg.H * cfg.D, cfg.c), generator=g, device=dev) / (cfg.H * cfg.D) ** 0.5).to(torch.bfloat16)
+        for _ in range(2):
+            pba.tri_out_proj_forward(o, w_o)
     elif args.profile == "pba4k":
         cfg = W.AttnConfig("pba4k", B=1, N=4096, H=16, D=64, dtype=torch.bfloat16, seed=4, mask="random5")
         q, k, v, bias, mask = W.attn_inputs(cfg, dev)
