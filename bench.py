@@ -40,6 +40,24 @@ def attn_flops(B, H, Nq, Nk, D) -> float:
     return 4.0 * B * H * Nq * Nk * D
 
 
+def tri_ceilings(N, H, D, ms_per_call, tensor_tflops, hbm_gbs, sm_mhz, n_sms) -> dict:
+    """The three ceilings of one triangle-attention call on a pair tensor of
+    N x N rows (one orientation, gate and lse written) and the measured call's
+    fraction of each: the tensor cores (4 N^3 H D FLOPs), HBM (q, k, v, gate
+    read and out written as bf16 [N,N,H,D], lse [N,N,H] fp32, bias [H,N,N]
+    bf16) and the exp2 unit (one exponential per score, N^3 H of them, at 16
+    per clock per SM).  frac = ceiling time / measured time."""
+    flops = 4.0 * N * N * N * H * D
+    nbytes = 5.0 * N * N * H * D * 2 + N * N * H * 4 + H * N * N * 2
+    exps = float(N) * N * N * H
+    floors = {"tensor": flops / (tensor_tflops * 1e12) * 1e3,
+              "hbm": nbytes / (hbm_gbs * 1e9) * 1e3,
+              "exp2": exps / (16.0 * n_sms * sm_mhz * 1e6) * 1e3}
+    return {"ms_per_call": ms_per_call, "floor_ms": floors,
+            "frac": {k: v / ms_per_call for k, v in floors.items()},
+            "flops_per_call": flops, "bytes_per_call": nbytes, "exps_per_call": exps}
+
+
 def attn_bytes(B, H, Nq, Nk, D, elt=2, mask=True) -> float:
     """Algorithmic HBM bytes of one pass: bias, Q, K, V read once, O and the
     log-sum-exp written once, the key mask read once."""
@@ -355,6 +373,10 @@ def main():
         "tri_attn_rows_per_s": tri_rows_per_s,
         "tri_attn_ms_per_call": sum(tri_ms) / len(tri_ms) / 2,
         "tri_attn_tflops": world * tri_flops * args.steps / (t_tri / 1e3) / 1e12,
+        "tri_attn_ceilings": tri_ceilings(tcfg.N, tcfg.H, tcfg.D, sum(tri_ms) / len(tri_ms) / 2,
+                                          peaks["bf16_tflops_sustained"], peaks["hbm_gbs"],
+                                          (clk.get("sm_mhz") or 1965.0) if isinstance(clk, dict) else 1965.0,
+                                          torch.cuda.get_device_properties(dev).multi_processor_count),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
                      "kernel": "pba_attn_sm100_kernel (pba_forward, large16k)",
