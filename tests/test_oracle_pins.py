@@ -437,6 +437,26 @@ def _pwa_problem(S=3, N=11, H=2, D=4, seed=0, mask_frac=0.3, neg_inf_frac=0.0):
     return v, bias, mask, gate
 
 
+def test_pwa_two_pass_reading_equals_one_pass():
+    """The kernels take the softmax in two passes (the row log-sum-exp, then
+    exp(b - lse) times the values); in exact arithmetic that is the one-pass
+    softmax the oracle computes, masks and -inf logits included."""
+    rng = np.random.default_rng(12)
+    S, N, H, D = 3, 20, 2, 4
+    v = rng.standard_normal((S, N, H, D))
+    b = rng.standard_normal((H, N, N)) * 2.0
+    b[1, 4, ::3] = -np.inf
+    mask = (rng.random(N) > 0.25).astype(np.uint8)
+    ref = oracle.pwa(v, b, mask)
+    logits = np.where(mask[None, None, :] != 0, b, -np.inf)
+    m = logits.max(axis=-1, keepdims=True)
+    lse = (m + np.log(np.exp(logits - m).sum(axis=-1, keepdims=True)))[..., 0]
+    w = np.exp(logits - lse[..., None])                     # second pass: normalised weights
+    o = np.einsum("hij,sjhd->sihd", w, v)
+    assert np.abs(lse - ref["lse"]).max() < 1e-12
+    assert np.abs(o - ref["o"]).max() < 1e-12
+
+
 def test_pwa_is_attention_with_zero_queries():
     v, bias, mask, _ = _pwa_problem(neg_inf_frac=0.1)
     r = oracle.pwa(v, bias, mask)
