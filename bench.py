@@ -65,6 +65,27 @@ def attn_bytes(B, H, Nq, Nk, D, elt=2, mask=True) -> float:
             (B * Nk if mask else 0))
 
 
+def roofline_entry(flops, nbytes, seconds, peaks, traffic, kernel):
+    """Roofline of one launch: the slower of the dense-bf16 floor (flops at the
+    burst tensor peak) and the HBM floor (algorithmic bytes at the copy
+    bandwidth) sets the bound; achieved and frac are in that bound's unit."""
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    tflops = flops / seconds / 1e12
+    gbs = nbytes / seconds / 1e9
+    if t_hbm >= t_tensor:
+        e = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": gbs / peaks["hbm_gbs"]}
+    else:
+        e = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+             "frac": tflops / peaks["bf16_tflops"]}
+    e.update({"traffic": traffic, "kernel": kernel, "algorithmic_bytes_per_launch": nbytes,
+              "flops_per_launch": flops, "floor_ms": {"tensor": t_tensor * 1e3, "hbm": t_hbm * 1e3},
+              "peak_source": peaks["source"], "tensor_frac": tflops / peaks["bf16_tflops"],
+              "tensor_frac_sustained": tflops / peaks["bf16_tflops_sustained"], "hbm_frac": gbs / peaks["hbm_gbs"]})
+    return e
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -204,34 +225,62 @@ def barrier(pg: bool):
 
 
 # ------------------------------------------------------------------ CPU oracle timing
-def oracle_sample(q, k, v, bias, mask, target_s=10.0, chunk_rows=1024):
-    """Times the fp64 oracle on sampled query rows of the large workload (all
-    16384 keys each), one chunk of rows per head round robin, until about
-    target_s seconds of oracle time.  Returns (TFLOP/s, threads, description,
-    seconds)."""
+ORACLE_CHUNK_ROWS = 1024
+
+
+def oracle_chunks(q, k, v, bias, mask, n_chunks, chunk_rows=ORACLE_CHUNK_ROWS, seed=77):
+    """Seeded chunks of query rows of the large workload, one head per chunk
+    round robin, each against all keys, converted to fp64 host arrays before
+    any timing (the conversion is not the oracle's work)."""
+    import numpy as np
+
+    H, N = q.shape[1], q.shape[2]
+    g = torch.Generator("cpu").manual_seed(seed)
+    ms = None if mask is None else mask.cpu().numpy().astype(np.uint8)
+    f64 = lambda t: np.ascontiguousarray(t.cpu().double().numpy())
+    kv = {}
+    for c in range(n_chunks):
+        h = c % H
+        rows = torch.randperm(N, generator=g)[:chunk_rows].to(q.device)
+        if h not in kv:
+            kv[h] = (f64(k[:, h:h + 1]), f64(v[:, h:h + 1]))
+        yield (f64(q[:, h:h + 1].index_select(2, rows)), kv[h][0], kv[h][1],
+               f64(bias[:, h:h + 1].index_select(2, rows)), ms)
+
+
+def time_oracle_chunk(chunk) -> float:
+    """Seconds of one oracle call on one chunk (all host cores)."""
     import oracle
 
-    H, N, D = q.shape[1], q.shape[2], q.shape[3]
-    g = torch.Generator("cpu").manual_seed(77)
-    flops, t, nrows, h = 0.0, 0.0, 0, 0
-    ms = None if mask is None else mask.cpu()
-    while t < target_s and nrows < 64 * chunk_rows:
-        rows = torch.randperm(N, generator=g)[:chunk_rows].to(q.device)
-        qs = q[:, h:h + 1].index_select(2, rows).cpu()
-        bs = bias[:, h:h + 1].index_select(2, rows).cpu()
-        ks, vs = k[:, h:h + 1].cpu(), v[:, h:h + 1].cpu()
-        t0 = time.perf_counter()
-        oracle.pba(qs, ks, vs, bs, ms)
-        t += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.pba(*chunk)
+    return time.perf_counter() - t0
+
+
+def oracle_sample(q, k, v, bias, mask, target_s=10.0, chunk_rows=ORACLE_CHUNK_ROWS):
+    """Times the fp64 oracle on sampled query rows of the large workload (all
+    16384 keys each), chunk by chunk, until about target_s seconds of oracle
+    time.  Returns (TFLOP/s, threads, description, seconds)."""
+    import oracle
+
+    N, D = q.shape[2], q.shape[3]
+    flops, t, nrows = 0.0, 0.0, 0
+    chunks = oracle_chunks(q, k, v, bias, mask, 256, chunk_rows)
+    for ch in chunks:
+        if t >= target_s:
+            break
+        t += time_oracle_chunk(ch)
         flops += attn_flops(1, 1, chunk_rows, N, D)
         nrows += chunk_rows
-        h = (h + 1) % H
     return (flops / t / 1e12, oracle.threads_used(),
             f"{nrows} query rows x {N} keys of large16k, {chunk_rows}-row chunks over the heads (fp64 oracle)", t)
 
 
 # ------------------------------------------------------------------ the reference arm
 def run_reference(args, world, rank):
+    """The oracle as the reference arm: each step is one 1024-row chunk of the
+    large workload's query rows against all keys (the chunking of the
+    cpu_baseline leg, so both report one oracle rate)."""
     if rank != 0:
         return 0
     import oracle
@@ -240,33 +289,23 @@ def run_reference(args, world, rank):
     cfg = W.LARGE16K
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     q, k, v, bias, mask = W.attn_inputs(cfg, dev)
-    # each step runs the oracle on a bounded sample of rows of this workload
     H, N, D = cfg.H, cfg.N, cfg.D
-    per_head = max(1, args.ref_rows // H)
-    g = torch.Generator("cpu").manual_seed(5)
-    sample = []
-    for h in range(H):
-        rows = torch.randperm(N, generator=g)[:per_head].to(q.device)
-        sample.append((q[:, h:h + 1].index_select(2, rows).cpu(), k[:, h:h + 1].cpu(), v[:, h:h + 1].cpu(),
-                       bias[:, h:h + 1].index_select(2, rows).cpu(), mask.cpu()))
-    del q, k, v, bias
-    flops_step = attn_flops(1, H, per_head, N, D)
-    for _ in range(args.warmup):
-        for s in sample[:1]:
-            oracle.pba(*s)
+    warm = max(1, args.warmup)
+    chunks = oracle_chunks(q, k, v, bias, mask, warm + args.steps)
     times = []
-    for _ in range(args.steps):
-        t0 = time.perf_counter()
-        for s in sample:
-            oracle.pba(*s)
-        times.append(time.perf_counter() - t0)
+    for c, ch in enumerate(chunks):  # each chunk converted before its timed call
+        t = time_oracle_chunk(ch)
+        if c >= warm:
+            times.append(t)
     total = sum(times)
+    flops_step = attn_flops(1, 1, ORACLE_CHUNK_ROWS, N, D)
     value = flops_step * args.steps / total / 1e12
     cores = oracle.threads_used()
-    desc = f"{per_head * H} query rows x {N} keys of large16k per step (fp64 oracle)"
+    desc = (f"{ORACLE_CHUNK_ROWS} query rows x {N} keys of large16k per step, one head per step round robin "
+            f"(fp64 oracle, {cores} threads)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "warmup": warm, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "large16k: pair-biased attention N=16384 H=16 D=64, 5% random key mask (sampled rows)",
                    "B": 1, "N": N, "H": H, "D": D},
@@ -287,10 +326,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "oproj1024", "pwa4k", "bwd4k"],
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "oproj1024", "pwa4k", "bwd4k",
+                                          "merge8k"],
                     default="none",
                     help="run one small case only (for ncu captures); prints no JSON line")
     args = ap.parse_args()
@@ -377,11 +416,8 @@ def main():
                                           peaks["bf16_tflops_sustained"], peaks["hbm_gbs"],
                                           (clk.get("sm_mhz") or 1965.0) if isinstance(clk, dict) else 1965.0,
                                           torch.cuda.get_device_properties(dev).multi_processor_count),
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": traffic,
-                     "kernel": "pba_attn_sm100_kernel (pba_forward, large16k)",
-                     "algorithmic_bytes_per_launch": nbytes, "peak_source": peaks["source"],
-                     "tensor_frac": (flops / avg_launch_s / 1e12) / peaks["bf16_tflops_sustained"]},
+        "roofline": roofline_entry(flops, nbytes, avg_launch_s, peaks, traffic,
+                                   "pba_attn_sm100_kernel (pba_forward, large16k)"),
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
@@ -390,6 +426,7 @@ def main():
     line["tri_out_proj"] = run_out_proj(args, pba, tcfg, dev, stream, pg, peaks)
     line["pwa"] = run_pwa(args, pba, dev, stream, pg, peaks, clk)
     line["backward"] = run_bwd(args, pba, dev, stream, pg, peaks)
+    line["ring8k"] = run_ring8k(args, pba, dev, stream, pg, peaks)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -551,6 +588,92 @@ def run_bwd(args, pba, dev, stream, pg, peaks):
                          "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
 
 
+def merge_bytes(P, rows, D, out_elt=2):
+    """Algorithmic bytes of softmax_merge: the P partials (O_p fp32, m_p, l_p)
+    read once, out and lse written once."""
+    return P * rows * (4 * D + 8) + rows * (out_elt * D + 4)
+
+
+def run_ring8k(args, pba, dev, stream, pg, peaks):
+    """The ring-step emulation on one GPU (ring8k: N=8192, H=16, D=64, bf16,
+    bias ~N(0,1), no mask): P=8 pba_partial calls over key blocks of 1024 in
+    randperm(8) order, each into its slot of one preallocated [8,B,H,N,D]
+    buffer, then softmax_merge into bf16 out and the lse.  The partials and the
+    merge are timed in their own CUDA-event regions; the merge also alone,
+    after an L2 flush each time (its 277 MB input otherwise partly sits in L2
+    from the last partial).  pba_forward at the same shape is timed beside."""
+    cfg = W.RING8K
+    q, k, v, bias, mask = W.attn_inputs(cfg, dev)
+    B, H, N, D, P = cfg.B, cfg.H, cfg.N, cfg.D, cfg.blocks
+    L = N // P
+    order = W.block_order(cfg)
+    o_parts = torch.empty((P, B, H, N, D), dtype=torch.float32, device=dev)
+    m_parts = torch.empty((P, B, H, N), dtype=torch.float32, device=dev)
+    l_parts = torch.empty_like(m_parts)
+    out = torch.empty((B, H, N, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    views = [(k[:, :, b * L:(b + 1) * L], v[:, :, b * L:(b + 1) * L], bias[..., b * L:(b + 1) * L]) for b in order]
+
+    def partials():
+        for slot, (kb, vb, bb) in enumerate(views):
+            pba.pba_partial(q, kb, vb, bb, None, o_parts[slot], m_parts[slot], l_parts[slot], stream=stream)
+
+    merge = lambda: pba.softmax_merge(o_parts, m_parts, l_parts, out_dtype=torch.bfloat16, out=out, lse=lse,
+                                      stream=stream)
+    fwd_out, fwd_lse = torch.empty_like(out), torch.empty_like(lse)
+    fwd = lambda: pba.pba_forward(q, k, v, bias, None, fwd_out, fwd_lse, stream=stream)
+    for _ in range(3):
+        partials()
+        merge()
+        fwd()
+    barrier(pg)
+    steps = max(3, args.steps // 4)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        ev[i][0].record(stream)
+        partials()
+        ev[i][1].record(stream)
+        merge()
+        ev[i][2].record(stream)
+    fs, fe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fs.record(stream)
+    for _ in range(steps):
+        fwd()
+    fe.record(stream)
+    # the merge alone, L2 flushed before each call
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    mev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        mev[i][0].record(stream)
+        merge()
+        mev[i][1].record(stream)
+    barrier(pg)
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("a ring-step kernel recorded a device error")
+    part_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev), pg) / steps
+    merge_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev), pg) / steps
+    merge_cold_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in mev), pg) / steps
+    fwd_ms = max_over_ranks(fs.elapsed_time(fe), pg) / steps
+    flops = attn_flops(B, H, N, N, D)
+    # partials: every block reads its bias columns, Q, its K/V block; writes O_p fp32, m_p, l_p
+    part_bytes = B * H * N * N * 2 + P * B * H * N * D * 2 + 2 * B * H * N * D * 2 + P * B * H * N * (4 * D + 8)
+    mbytes = merge_bytes(P, B * H * N, D)
+    return {"partials_ms": part_ms, "merge_ms_in_step": merge_ms, "merge_ms_l2_flushed": merge_cold_ms,
+            "pba_forward_ms_same_shape": fwd_ms, "steps": steps, "gpu_launches": steps * (P + 1),
+            "workload": f"ring8k: N={N} H={H} D={D} bf16, P={P} key blocks of {L} in order {order}, "
+                        f"partials into one preallocated [P,B,H,N,D] buffer, then softmax_merge",
+            "partials_tflops": flops / (part_ms / 1e3) / 1e12,
+            "partials_roofline": roofline_entry(flops, part_bytes, part_ms / 1e3, peaks, None,
+                                                "pba_attn_sm100_kernel (pba_partial x 8)"),
+            "merge_roofline": {"bound": "hbm", "achieved": mbytes / (merge_cold_ms / 1e3) / 1e9,
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": mbytes / (merge_cold_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                               "algorithmic_bytes_per_call": mbytes, "kernel": "softmax_merge_kernel",
+                               "peak_source": peaks["source"],
+                               "in_step_gbs": mbytes / (merge_ms / 1e3) / 1e9}}
+
+
 def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops):
     """Same metric through the public call with the inputs starting in pinned
     host memory and the outputs read back each step."""
@@ -590,10 +713,26 @@ def run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, fl
 def run_profile_case(args, pba, dev):
     """One small case for ncu, each kernel launched twice (a warm-up launch,
     then the captured one): pba4k = pba_forward at N=4096 (bias 512 MB, larger
-    than L2); tri512 = triangle attention N=512 both orientations; proj1024 /
+    than L2); merge8k = softmax_merge of the ring8k partials (L2 flushed
+    before each merge); tri512 = triangle attention N=512 both orientations; proj1024 /
     oproj1024 = the input / output projections at tri1024; pwa4k = pwa_forward;
     bwd4k = pba_backward at N=4096, H=4."""
-    if args.profile == "bwd4k":
+    if args.profile == "merge8k":
+        cfg = W.RING8K
+        q, k, v, bias, _ = W.attn_inputs(cfg, dev)
+        P, L = cfg.blocks, cfg.N // cfg.blocks
+        o_parts = torch.empty((P,) + tuple(q.shape), dtype=torch.float32, device=dev)
+        m_parts = torch.empty((P,) + tuple(q.shape[:3]), dtype=torch.float32, device=dev)
+        l_parts = torch.empty_like(m_parts)
+        for slot, b in enumerate(W.block_order(cfg)):
+            sl = slice(b * L, (b + 1) * L)
+            pba.pba_partial(q, k[:, :, sl], v[:, :, sl], bias[..., sl], None, o_parts[slot], m_parts[slot],
+                            l_parts[slot])
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for i in range(2):
+            flush.fill_(i)
+            pba.softmax_merge(o_parts, m_parts, l_parts, out_dtype=torch.bfloat16)
+    elif args.profile == "bwd4k":
         q, k, v, bias, mask = W.random_attn(1, 4, 4096, 4096, 64, seed=12, device=dev, mask_frac=0.05)
         out, lse = pba.pba_forward(q, k, v, bias, mask)
         dout = torch.randn(q.shape, generator=torch.Generator(dev.type).manual_seed(13), device=dev).to(torch.bfloat16)

@@ -190,6 +190,39 @@ def test_tri1024_sampled_lines(cuda_device, ending):
     _tri_lines_check(f"tri1024 ending={ending}", cfg, q, k, v, g, bias, ending, lines)
 
 
+@pytest.mark.parametrize("N,H,D", [(136, 4, 32), (200, 2, 64)])
+@pytest.mark.parametrize("ending", [False, True])
+@pytest.mark.parametrize("masked", [False, True])
+def test_tri_key_tail_and_pair_mask(cuda_device, N, H, D, ending, masked):
+    """Triangle attention with N % 128 != 0: the last key tile runs past the
+    end of every line and the last query tile is partly filled.  Both
+    orientations, with and without a random pair mask, against the oracle's
+    explicit index formulas.  With the mask, one line has every key masked
+    and must give out = 0 and lse = -inf."""
+    cfg = W.TriConfig(f"tail{N}", N=N, c=32, H=H, D=D, seed=N + (1 if ending else 0))
+    q, k, v, g, bias = W.tri_inputs(cfg, cuda_device)
+    dead = 3
+    pm = None
+    if masked:
+        gen = torch.Generator("cuda").manual_seed(N * 3 + int(ending))
+        pm = (torch.rand((N, N), generator=gen, device=cuda_device) > 0.25).to(torch.uint8)
+        # the keys of line `dead`: row dead (starting node) or column dead (ending node)
+        if ending:
+            pm[:, dead] = 0
+        else:
+            pm[dead, :] = 0
+    out, lse = pba.tri_attn_forward(q, k, v, bias, g, pm, "ending" if ending else "starting")
+    lines = sorted({0, dead, 127, 128, N // 2, N - 1})
+    ref = oracle.tri_attn(q, k, v, bias, g, pm, ending=ending, lines=lines)
+    o_sel = out[:, lines].transpose(0, 1) if ending else out[lines]
+    l_sel = lse[:, lines].transpose(0, 1) if ending else lse[lines]
+    _cmp(f"tri tail N={N} D={D} ending={ending} masked={masked}", o_sel, l_sel, ref)
+    if masked:
+        o_dead = out[:, dead] if ending else out[dead]
+        l_dead = lse[:, dead] if ending else lse[dead]
+        assert torch.all(o_dead == 0) and torch.all(l_dead == -math.inf)
+
+
 # ------------------------------------------------------------------ shapes and edge cases
 @pytest.mark.parametrize("Nq,Nk,D,mask_frac", [
     (1, 1, 64, 0.0), (17, 17, 64, 0.0), (100, 100, 32, 0.2), (1000, 1000, 64, 0.05), (1025, 1025, 32, 0.0),
@@ -213,10 +246,10 @@ def test_shapes(cuda_device, Nq, Nk, D, mask_frac, dtype):
 @pytest.mark.parametrize("D", [32, 64])
 @pytest.mark.parametrize("scale", [0.125, 0.25, 0.13, 0.3])
 def test_bias_modes(cuda_device, D, scale):
-    """A softmax scale that is a power of two has the tensor core add the bias
-    (scores S = Q K^T + bias / scale, the mask as a rank-1 MMA); any other
-    scale has the softmax warps add it.  Both against the oracle, masked and
-    ragged, forward and partial."""
+    """The softmax warps add the bias to tau * (Q K^T) for every scale: powers
+    of two (0.125, 0.25, where tau * s is exact) and others (0.13, 0.3).
+    Against the oracle, masked and ragged, forward and partial, then unmasked
+    whole tiles (no mask words)."""
     q, k, v, bias, mask = W.random_attn(2, 3, 333, 421, D, seed=int(scale * 1000) + D, device=cuda_device,
                                         mask_frac=0.1)
     out, lse = pba.pba_forward(q, k, v, bias, mask, softmax_scale=scale)
@@ -224,7 +257,7 @@ def test_bias_modes(cuda_device, D, scale):
     _cmp(f"bias mode D={D} scale={scale}", out, lse, ref)
     o_p, m_p, l_p = pba.pba_partial(q, k, v, bias, mask, softmax_scale=scale)
     _cmp(f"bias mode partial D={D} scale={scale}", o_p, m_p + torch.log(l_p), ref)
-    # unmasked whole tiles: no mask MMA
+    # unmasked whole tiles: the kernel instance without mask words
     q, k, v, bias, _ = W.random_attn(1, 2, 256, 512, D, seed=D + 1, device=cuda_device)
     out, lse = pba.pba_forward(q, k, v, bias, softmax_scale=scale)
     _cmp(f"bias mode unmasked D={D} scale={scale}", out, lse, oracle.pba(q, k, v, bias, softmax_scale=scale))
@@ -248,9 +281,10 @@ def _padded_clone(b):
 
 @pytest.mark.parametrize("D,scale", [(64, None), (32, 0.25), (32, None), (64, 0.1)])
 def test_minus_inf_bias_and_fully_masked_rows(cuda_device, D, scale):
-    """-inf bias entries exclude their keys.  With a power-of-two scale the
-    first pass (bias added by the tensor core) turns them into NaN rows, and
-    the re-run recomputes those units; the result must not show it."""
+    """-inf bias entries exclude their keys exactly like masked keys: a row
+    with no valid key gives O = 0 and lse = -inf, scattered and tile-sized
+    -inf regions drop out, and no NaN appears, with the default scale and a
+    power-of-two scale alike."""
     q, k, v, bias, mask = W.random_attn(1, 2, 600, 260, D, seed=9, device=cuda_device, mask_frac=0.05)
     bias = _padded_clone(bias)
     bias[0, 0, 5, :] = -math.inf              # row with no valid key
