@@ -260,6 +260,38 @@ PBA_API pba_status pba_backward(const pba_attn_desc *desc, const void *q, const 
                                 const void *dout, float *dq, float *dk, float *dv, void *dbias, float *delta,
                                 void *stream);
 
+/*
+ * pba_backward_noalloc -- pba_backward for callers that cannot allocate
+ * device memory.  No counterpart on the pages: it exists for callers that
+ * hold only the tensors they were handed and no device allocator of their
+ * own (a plugin inside another runtime's memory manager, a C host program
+ * that links this library alone), or that must not call cudaMalloc or
+ * cudaFree on their path because those calls can synchronise the device and
+ * stall the work of other streams.
+ *
+ * Same arguments, checks, results and launches as pba_backward, without the
+ * `delta` argument: the per-row Delta = rowsum(dout * out) that pba_backward
+ * writes to a caller buffer goes to a fixed array of
+ * PBA_BWD_NOALLOC_MAX_ROWS floats (4 MiB) inside the library, which every
+ * GPU that loads the library holds until the process exits.  The call
+ * allocates nothing.
+ *   - B * H * Nq above PBA_BWD_NOALLOC_MAX_ROWS: PBA_ERR_INVALID_ARG before
+ *     anything else (use pba_backward with a delta buffer of your own).
+ *   - The first call on a device looks up that device's address of the array
+ *     (with the device current); make that first call before any stream
+ *     capture.  Every later call on the device reuses the address.
+ *   - Every call on a device shares the one array and leaves its Delta in it.
+ *     Nothing in it must start at zero: each call writes every row it reads
+ *     before reading it.  Calls whose kernels overlap on the GPU (different
+ *     streams, no ordering between them) race on the array and may compute
+ *     wrong gradients: order them on one stream or with events.
+ */
+#define PBA_BWD_NOALLOC_MAX_ROWS 1048576
+PBA_API pba_status pba_backward_noalloc(const pba_attn_desc *desc, const void *q, const void *k, const void *v,
+                                        const void *bias, const uint8_t *key_mask, const void *out,
+                                        const float *lse, const void *dout, float *dq, float *dk, float *dv,
+                                        void *dbias, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 PBA_API const char *pba_status_string(pba_status status);
 

@@ -23,6 +23,7 @@ import torch
 __all__ = [
     "PbaError", "PBA_OK", "PBA_ERR_INVALID_ARG", "PBA_ERR_UNSUPPORTED", "PBA_ERR_CUDA", "PBA_ERR_TIMEOUT",
     "library_path", "load_library", "pba_forward", "pba_partial", "softmax_merge", "tri_attn_forward", "tri_proj_forward", "tri_out_proj_forward", "pwa_forward", "pba_backward",
+    "pba_backward_noalloc", "PBA_BWD_NOALLOC_MAX_ROWS",
     "pba_last_device_error", "pba_set_wait_timeout_ns", "pba_selftest_wait_timeout", "pba_selftest_exp2",
     "pba_status_string",
 ]
@@ -30,6 +31,8 @@ __all__ = [
 PBA_OK, PBA_ERR_INVALID_ARG, PBA_ERR_UNSUPPORTED, PBA_ERR_CUDA, PBA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 PBA_BF16, PBA_F32 = 0, 1
 PBA_TRI_STARTING, PBA_TRI_ENDING = 0, 1
+# rows (B * H * Nq) of the fixed Delta array of pba_backward_noalloc (include/pba.h)
+PBA_BWD_NOALLOC_MAX_ROWS = 1048576
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -89,6 +92,8 @@ def load_library() -> ctypes.CDLL:
     lib.pwa_forward.restype = st
     lib.pba_backward.argtypes = [desc_p] + [_p] * 14
     lib.pba_backward.restype = st
+    lib.pba_backward_noalloc.argtypes = [desc_p] + [_p] * 13
+    lib.pba_backward_noalloc.restype = st
     lib.pba_status_string.argtypes = [st]
     lib.pba_status_string.restype = ctypes.c_char_p
     lib.pba_last_device_error.argtypes = [_p]
@@ -385,6 +390,42 @@ def pba_backward(q, k, v, bias, key_mask, out, lse, dout, softmax_scale=None, st
                                                        _ptr(dk), _ptr(dv), _ptr(dbias), _ptr(delta),
                                                        _stream(stream)))
     return dq, dk, dv, dbias, delta
+
+
+def pba_backward_noalloc(q, k, v, bias, key_mask, out, lse, dout, softmax_scale=None, stream=None, grads=None):
+    """pba_backward through the entry point that allocates nothing on the
+    device: Delta goes to the library's fixed array (B*H*Nq rows at most,
+    PBA_BWD_NOALLOC_MAX_ROWS), so no delta buffer is passed.  For callers
+    that cannot allocate device memory; ``grads`` = (dq, dk, dv, dbias)
+    preallocated by the caller (allocated here when None).  Calls that
+    overlap on the GPU race on the shared array.  Returns dq, dk, dv, dbias."""
+    for n, t in (("out", out), ("dout", dout)):
+        _cuda(n, t, torch.bfloat16)
+    _cuda("lse", lse, torch.float32)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse)):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, H, Nq, D = q.shape
+    Nk = k.shape[2]
+    if out.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, H, Nq):
+        raise ValueError("out and dout must be [B,H,Nq,D], lse [B,H,Nq]")
+    if grads is None:
+        grads = (torch.empty(q.shape, dtype=torch.float32, device=q.device),
+                 torch.empty(k.shape, dtype=torch.float32, device=q.device),
+                 torch.empty(v.shape, dtype=torch.float32, device=q.device),
+                 torch.empty((B, H, Nq, Nk), dtype=torch.bfloat16, device=q.device))
+    dq, dk, dv, dbias = grads
+    for n, t, dt, shape in (("dq", dq, torch.float32, q.shape), ("dk", dk, torch.float32, k.shape),
+                            ("dv", dv, torch.float32, v.shape), ("dbias", dbias, torch.bfloat16, (B, H, Nq, Nk))):
+        _cuda(n, t, dt)
+        if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous {tuple(shape)} tensor")
+    d = _desc(q, k, v, bias, key_mask, out.stride()[:3] if out.dim() == 4 else None, lse.stride(), softmax_scale)
+    _check("pba_backward_noalloc",
+           load_library().pba_backward_noalloc(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(bias),
+                                               _ptr(key_mask), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk),
+                                               _ptr(dv), _ptr(dbias), _stream(stream)))
+    return dq, dk, dv, dbias
 
 
 def pba_last_device_error(stream=None) -> int:

@@ -809,6 +809,55 @@ pba_status pba_backward(const pba_attn_desc *d, const void *q, const void *k, co
   return PBA_OK;
 }
 
+}  // extern "C"
+
+// ------------------------------------------------------------ pba_backward_noalloc
+// The Delta rows of pba_backward_noalloc: a fixed array in every GPU that
+// loads the library, shared by all its calls on that device.
+static __device__ __align__(256) float g_bwd_noalloc_delta[PBA_BWD_NOALLOC_MAX_ROWS];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float *g_noalloc_delta_ptr[kNoallocMaxDevices] = {};
+
+// Device address of g_bwd_noalloc_delta on the current device.  In host code
+// the array's name is a host-side stand-in, not a device address, so it is
+// looked up once per device (with that device current) and kept.
+pba_status noalloc_delta(float **ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PBA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return PBA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_delta_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_noalloc_delta) != cudaSuccess || p == nullptr) return PBA_ERR_CUDA;
+    g_noalloc_delta_ptr[dev] = static_cast<float *>(p);
+  }
+  *ptr = g_noalloc_delta_ptr[dev];
+  return PBA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pba_status pba_backward_noalloc(const pba_attn_desc *d, const void *q, const void *k, const void *v,
+                                const void *bias, const uint8_t *key_mask, const void *out, const float *lse,
+                                const void *dout, float *dq, float *dk, float *dv, void *dbias, void *stream) {
+  if (d == nullptr || d->B < 1 || d->H < 1 || d->Nq < 0) return PBA_ERR_INVALID_ARG;
+  const int64_t cap = PBA_BWD_NOALLOC_MAX_ROWS;
+  if (d->B > cap || d->H > cap || d->Nq > cap || d->B * d->H > cap || d->B * d->H * d->Nq > cap)
+    return PBA_ERR_INVALID_ARG;  // more rows than the fixed Delta array holds
+  pba_status s = check_device();
+  if (s != PBA_OK) return s;
+  float *delta = nullptr;
+  s = noalloc_delta(&delta);
+  if (s != PBA_OK) return s;
+  return pba_backward(d, q, k, v, bias, key_mask, out, lse, dout, dq, dk, dv, dbias, delta, stream);
+}
+
 const char *pba_status_string(pba_status status) {
   switch (status) {
     case PBA_OK:
