@@ -522,6 +522,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         for (int c = 0; c < kBN / 32; ++c)
           tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sreg[c * 32]));
         tmem_wait_ld();
+        reg_fence(sreg);
         tc_fence_before_sync();
         mbar_arrive(&bars[L::kBarSFree + w]);
 
@@ -561,8 +562,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
             }
           }
         }
-        mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
-
         // tile maximum: eight independent chains
         float m8[8];
 #pragma unroll
@@ -570,6 +569,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
 #pragma unroll
         for (int i = 8; i < kBN / 2; ++i) m8[i & 7] = max3f(m8[i & 7], x[i].x, x[i].y);
         const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        // The bias slot is released under a condition on mx, which depends on
+        // every bias value of the tile: the arrive cannot issue before all of
+        // the slot's shared-memory loads have returned, so the next TMA write
+        // into the slot cannot overtake one still in flight.  (The pattern
+        // never occurs: no maximum is this NaN.)
+        if (__float_as_uint(mx) != 0x7FC0DEADu) mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
         m_true = fmaxf(m_true, mx);
         const bool need = mx > m_cur + kRescaleThreshold;
         float alpha = 1.f;
@@ -608,6 +613,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
               uint32_t o[32];
               tmem_ld32(tO + c, o);
               tmem_wait_ld();
+              reg_fence(o);
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
               tmem_st32(tO + c, o);
@@ -631,6 +637,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         uint32_t r[32];
         tmem_ld32(tO + c, r);
         tmem_wait_ld();
+        reg_fence(r);
 #pragma unroll
         for (int e = 0; e < 32; ++e) o[c + e] = __uint_as_float(r[e]);
       }

@@ -362,6 +362,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
         tmem_ld32(tmem + lane_base + L::kColDP + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&dpv[0]));
         tmem_ld32(tmem + lane_base + L::kColDP + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dpv[32]));
         tmem_wait_ld();
+        reg_fence(sv);
+        reg_fence(dpv);
         // S and dP are in registers: the next step's S, dP may overwrite them
         // once both warpgroups have arrived
         tc_fence_before_sync();
@@ -483,6 +485,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
           uint32_t v[32];
           tmem_ld32(tmem + lane_base + col + c, v);
           tmem_wait_ld();
+          reg_fence(v);
           if (r < nrows) {
             float4 *o = reinterpret_cast<float4 *>(dst + ((int64_t(b) * p.H + h) * nrows + r) * D + c);
 #pragma unroll

@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(kOprojThreads, 1) pba_oproj_sm100_kernel(const
         uint32_t a[32];
         tmem_ld32(tmem + lane_base + b * kC + 32 * ch, a);
         tmem_wait_ld();
+        reg_fence(a);
         if (ch + 1 == kC / 32) {
           tc_fence_before_sync();
           mbar_arrive(&bars[L::kBarAccEmpty + b]);  // this accumulator is free

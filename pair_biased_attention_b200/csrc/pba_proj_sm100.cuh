@@ -246,6 +246,8 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
           tmem_ld32(tmem + lane_base + 256 * hf + 32 * cc, a[0]);
           tmem_ld32(tmem + lane_base + 256 * hf + 32 * (cc + 1), a[1]);
           tmem_wait_ld();
+          reg_fence(a[0]);
+          reg_fence(a[1]);
           if (cc == 6) {
             tc_fence_before_sync();
             mbar_arrive(&bars[L::kBarAccEmpty + hf]);  // this half of Tensor Memory is free

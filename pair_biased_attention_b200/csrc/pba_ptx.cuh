@@ -302,6 +302,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 #undef PBA_W8
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// tcgen05.ld fills its destination registers asynchronously: they hold the
+// loaded values only after tcgen05.wait::ld.  The compiler does not know that
+// and may move arithmetic on those registers ahead of the wait (a memory
+// clobber does not order register-only work).  reg_fence passes each register
+// through an empty volatile asm placed after the wait, so every later use
+// depends on an instruction that follows the wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+__device__ __forceinline__ void reg_fence(uint32_t &r) { asm volatile("" : "+r"(r)); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Warpgroup register reallocation (all four warps of a warpgroup execute it).

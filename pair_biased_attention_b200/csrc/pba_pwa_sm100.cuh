@@ -462,7 +462,6 @@ __global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __g
             pk[i] = pack_bf16x2(pv.x, pv.y);
           }
         }
-        mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
         // the weight buffer of this tile was last read by the products of tile gt - 2
         const int b = gt & 1;
         if (gt >= 2) {
@@ -472,6 +471,11 @@ __global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __g
           tc_fence_after_sync();
         }
         tmem_st16(tP + b * (kPwaBN / 2), pk);
+        // The bias slot is released only after the store above, which takes
+        // every weight of the tile and so cannot issue before all of the
+        // slot's shared-memory loads have returned; released any earlier, the
+        // next TMA write into the slot could overtake a load still in flight.
+        mbar_arrive(&bars[L::kBarBiasEmpty + slot]);
         tmem_wait_st();
         tc_fence_before_sync();
         mbar_arrive(&bars[L::kBarPFull + b]);
@@ -505,6 +509,7 @@ __global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __g
         uint32_t r[32];
         tmem_ld32(tO + cc * 32, r);
         tmem_wait_ld();
+        reg_fence(r);
         if (cc + 1 == kChunks) {
           tc_fence_before_sync();
           mbar_arrive(&bars[L::kBarOFree]);  // O is in registers

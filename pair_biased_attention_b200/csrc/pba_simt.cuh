@@ -112,8 +112,11 @@ __global__ void __launch_bounds__(128) pba_attn_f32_kernel(const SimtParams p) {
 
 // Tiled-softmax merge.  Each thread owns 4 consecutive elements of one row
 // (D/4 threads per row); the per-row maxima and weights are recomputed by each
-// of those threads from the m_p, l_p values (cached loads).
-template <bool kOutBf16>
+// of those threads from the m_p, l_p values (cached loads).  kUnrollP > 0
+// handles P <= kUnrollP with every partial's loads issued before any of the
+// arithmetic (P independent 16-byte loads in flight per thread, which the
+// bandwidth-bound pass needs); kUnrollP = 0 is the loop for any P.
+template <bool kOutBf16, int kUnrollP>
 __global__ void __launch_bounds__(256) softmax_merge_kernel(int P, int64_t rows, int D, const float *o_parts,
                                                             const float *m_parts, const float *l_parts, void *out,
                                                             float *lse) {
@@ -124,24 +127,56 @@ __global__ void __launch_bounds__(256) softmax_merge_kernel(int P, int64_t rows,
     const int64_t r = idx / tpr;
     const int c = int(idx - r * tpr);
     float M = -INFINITY;
-    for (int pp = 0; pp < P; ++pp) {
-      const float lp = __ldg(l_parts + int64_t(pp) * rows + r);
-      const float mp = __ldg(m_parts + int64_t(pp) * rows + r);
-      if (lp > 0.f && mp > M) M = mp;
-    }
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float Lsum = 0.f;
-    if (M != -INFINITY) {
+    if (kUnrollP > 0) {
+      float lp[kUnrollP > 0 ? kUnrollP : 1], mp[kUnrollP > 0 ? kUnrollP : 1];
+      float4 ov[kUnrollP > 0 ? kUnrollP : 1];
+#pragma unroll
+      for (int pp = 0; pp < kUnrollP; ++pp) {
+        if (pp < P) {
+          lp[pp] = __ldg(l_parts + int64_t(pp) * rows + r);
+          mp[pp] = __ldg(m_parts + int64_t(pp) * rows + r);
+          ov[pp] = __ldcs(reinterpret_cast<const float4 *>(o_parts + (int64_t(pp) * rows + r) * D) + c);
+        } else {
+          lp[pp] = 0.f;
+          mp[pp] = -INFINITY;
+          ov[pp] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int pp = 0; pp < kUnrollP; ++pp)
+        if (lp[pp] > 0.f && mp[pp] > M) M = mp[pp];
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int pp = 0; pp < kUnrollP; ++pp) {
+          if (!(lp[pp] > 0.f)) continue;  // an empty block adds nothing, whatever its O holds
+          const float wgt = lp[pp] * expf(mp[pp] - M);
+          Lsum += wgt;
+          acc.x = fmaf(wgt, ov[pp].x, acc.x);
+          acc.y = fmaf(wgt, ov[pp].y, acc.y);
+          acc.z = fmaf(wgt, ov[pp].z, acc.z);
+          acc.w = fmaf(wgt, ov[pp].w, acc.w);
+        }
+      }
+    } else {
       for (int pp = 0; pp < P; ++pp) {
         const float lp = __ldg(l_parts + int64_t(pp) * rows + r);
-        if (!(lp > 0.f)) continue;
-        const float wgt = lp * expf(__ldg(m_parts + int64_t(pp) * rows + r) - M);
-        const float4 ov = __ldg(reinterpret_cast<const float4 *>(o_parts + (int64_t(pp) * rows + r) * D) + c);
-        Lsum += wgt;
-        acc.x = fmaf(wgt, ov.x, acc.x);
-        acc.y = fmaf(wgt, ov.y, acc.y);
-        acc.z = fmaf(wgt, ov.z, acc.z);
-        acc.w = fmaf(wgt, ov.w, acc.w);
+        const float mp = __ldg(m_parts + int64_t(pp) * rows + r);
+        if (lp > 0.f && mp > M) M = mp;
+      }
+      if (M != -INFINITY) {
+        for (int pp = 0; pp < P; ++pp) {
+          const float lp = __ldg(l_parts + int64_t(pp) * rows + r);
+          if (!(lp > 0.f)) continue;
+          const float wgt = lp * expf(__ldg(m_parts + int64_t(pp) * rows + r) - M);
+          const float4 ov = __ldcs(reinterpret_cast<const float4 *>(o_parts + (int64_t(pp) * rows + r) * D) + c);
+          Lsum += wgt;
+          acc.x = fmaf(wgt, ov.x, acc.x);
+          acc.y = fmaf(wgt, ov.y, acc.y);
+          acc.z = fmaf(wgt, ov.z, acc.z);
+          acc.w = fmaf(wgt, ov.w, acc.w);
+        }
       }
     }
     const float inv = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
