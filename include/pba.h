@@ -298,7 +298,10 @@ PBA_API const char *pba_status_string(pba_status status);
 /*
  * pba_last_device_error -- synchronises `stream`, then returns and clears the
  * device error word of the current device (PBA_OK if no kernel recorded an
- * error since the last call; PBA_ERR_TIMEOUT if a bounded wait ran out).
+ * error since the last call; PBA_ERR_TIMEOUT if a bounded wait ran out).  The
+ * read and the clear are one atomic exchange on the device, so an error that
+ * a kernel on another stream records meanwhile is reported by this call or
+ * the next, never lost.  Launches one single-thread kernel on `stream`.
  * Returns PBA_ERR_CUDA if the synchronisation itself failed.
  */
 PBA_API pba_status pba_last_device_error(void *stream);

@@ -24,6 +24,13 @@
 // cleared by pba_last_device_error().
 __device__ int g_pba_err = 0;
 
+// pba_last_device_error takes the word with one atomic exchange on the device
+// (so an error recorded between a read and a separate clear is never lost)
+// into one of these slots; concurrent callers use different slots.
+constexpr int kErrTakeSlots = 64;
+__device__ int g_pba_err_taken[kErrTakeSlots];
+__global__ void pba_take_error_kernel(int slot) { g_pba_err_taken[slot] = atomicExch(&g_pba_err, 0); }
+
 namespace {
 
 constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;
@@ -62,6 +69,22 @@ int *device_error_word() {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// One-time per-device kernel set-up (the dynamic shared memory limit is a
+// per-device attribute of a kernel): `setup` runs once for each device it is
+// called on, with that device current, and its result is kept per device.
+constexpr int kMaxDevices = 64;
+struct PerDeviceOnce {
+  std::once_flag flag[kMaxDevices];
+  cudaError_t err[kMaxDevices] = {};
+};
+template <typename F>
+cudaError_t once_per_device(PerDeviceOnce &o, F &&setup) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::call_once(o.flag[dev], [&] { o.err[dev] = setup(); });
+  return o.err[dev];
+}
 
 constexpr int64_t kMaxI32 = 2147483647;
 
@@ -117,17 +140,17 @@ template <int D, bool kBiasT, int kEpi, bool kGate, bool kMasked>
 cudaError_t launch_tc(const pba::AttnParams &p, int grid, cudaStream_t stream) {
   using L = pba::AttnLayout<D>;
   auto kern = pba::pba_attn_sm100_kernel<D, kBiasT, kEpi, kGate, kMasked>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [&] {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
     // The kernel moves registers between its warpgroups with setmaxnreg; the
     // split must fit in what the block is launched with, or the increase
     // would wait forever.  Refuse to launch a build where it would not.
     cudaFuncAttributes fa;
-    if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+    if (e == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
         fa.numRegs * pba::kAttnThreads < pba::kRegSplitTotal)
-      attr_err = cudaErrorInvalidConfiguration;
+      e = cudaErrorInvalidConfiguration;
+    return e;
   });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kAttnThreads, L::kSmemAlloc, stream>>>(p);
@@ -375,11 +398,9 @@ pba_status attn_common(const pba_attn_desc *d, const void *q, const void *k, con
 template <int kH>
 cudaError_t launch_proj(const pba::ProjParams &p, int grid, cudaStream_t stream) {
   auto kern = pba::pba_proj_sm100_kernel<kH>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pba::ProjLayout::kSmemAlloc);
-  });
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once_per_device(
+      once, [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pba::ProjLayout::kSmemAlloc); });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kProjThreads, pba::ProjLayout::kSmemAlloc, stream>>>(p);
   return cudaGetLastError();
@@ -389,11 +410,9 @@ template <int kC>
 cudaError_t launch_oproj(const pba::OprojParams &p, int grid, cudaStream_t stream) {
   using L = pba::OprojLayout<kC>;
   auto kern = pba::pba_oproj_sm100_kernel<kC>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
-  });
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once_per_device(
+      once, [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc); });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kOprojThreads, L::kSmemAlloc, stream>>>(p);
   return cudaGetLastError();
@@ -404,11 +423,9 @@ template <int D, bool kGate, bool kMasked>
 cudaError_t launch_pwa(const pba::PwaParams &p, int grid, cudaStream_t stream) {
   using L = pba::PwaLayout<D>;
   auto kern = pba::pba_pwa_sm100_kernel<D, kGate, kMasked>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
-  });
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once_per_device(
+      once, [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc); });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kPwaThreads, L::kSmemAlloc, stream>>>(p);
   return cudaGetLastError();
@@ -426,15 +443,15 @@ template <int D, bool kB>
 cudaError_t launch_bwd(const pba::BwdParams &p, int grid, cudaStream_t stream) {
   using L = pba::BwdLayout<D>;
   auto kern = pba::pba_bwd_sm100_kernel<D, kB>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once_per_device(once, [&] {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
     // the register split must fit in what the block is launched with (see launch_tc)
     cudaFuncAttributes fa;
-    if (attr_err == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+    if (e == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
         fa.numRegs * pba::kBwdThreads < pba::kBwdRegSplitTotal)
-      attr_err = cudaErrorInvalidConfiguration;
+      e = cudaErrorInvalidConfiguration;
+    return e;
   });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, pba::kBwdThreads, L::kSmemAlloc, stream>>>(p);
@@ -879,14 +896,18 @@ const char *pba_status_string(pba_status status) {
   return "PBA_ERR_UNKNOWN";
 }
 
-pba_status pba_last_device_error(void *stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PBA_ERR_CUDA;
+pba_status pba_last_device_error(void *stream_ptr) {
+  static std::atomic<unsigned> next_slot{0};
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PBA_ERR_CUDA;
+  const int slot = int(next_slot.fetch_add(1) % kErrTakeSlots);
+  pba_take_error_kernel<<<1, 1, 0, stream>>>(slot);
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_pba_err, sizeof(int)) != cudaSuccess) return PBA_ERR_CUDA;
-  if (v != 0) {
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(g_pba_err, &zero, sizeof(int)) != cudaSuccess) return PBA_ERR_CUDA;
-  }
+  if (cudaGetLastError() != cudaSuccess ||
+      cudaMemcpyFromSymbolAsync(&v, g_pba_err_taken, sizeof(int), slot * sizeof(int), cudaMemcpyDeviceToHost,
+                                stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return PBA_ERR_CUDA;
   return static_cast<pba_status>(v);
 }
 

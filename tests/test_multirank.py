@@ -51,10 +51,12 @@ def test_single_rank_needs_no_group():
 
 
 # ---------------------------------------------------------------- ring attention schedule (gloo, CPU)
-def _oracle_partial(q, k, v, bias, key_mask, softmax_scale=None, stream=None):
+def _oracle_partial(q, k, v, bias, key_mask, o_part, m_part, l_part, softmax_scale=None, stream=None):
     import oracle
     r = oracle.pba_partial(q, k, v, bias, key_mask, softmax_scale)
-    return tuple(torch.from_numpy(r[n]) for n in ("o", "m", "l"))
+    for dst, n in ((o_part, "o"), (m_part, "m"), (l_part, "l")):
+        dst.copy_(torch.from_numpy(r[n]))
+    return o_part, m_part, l_part
 
 
 def _oracle_merge(o, m, l, out_dtype=None, stream=None):
