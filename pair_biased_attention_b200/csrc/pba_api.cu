@@ -495,8 +495,8 @@ pba_status softmax_merge(int32_t P, int64_t rows, int64_t D, const float *o_part
   int64_t grid = (total + 255) / 256;
   const int64_t cap = int64_t(sms) * 8;  // a few resident blocks per SM, grid-stride beyond
   if (grid > cap) grid = cap;
-  // P up to 8 (the ring steps of one node) unrolled with all loads up front; larger P loops
   const bool bf = out_dtype == PBA_BF16;
+  // P up to 8 (the ring steps of one node) unrolled with all loads up front; larger P loops
   if (P <= 4)
     (bf ? pba::softmax_merge_kernel<true, 4> : pba::softmax_merge_kernel<false, 4>)<<<int(grid), 256, 0, stream>>>(
         P, rows, int(D), o_parts, m_parts, l_parts, out, lse);

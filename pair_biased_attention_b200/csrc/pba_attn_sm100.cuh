@@ -674,8 +674,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
             for (int e = 0; e < 4; ++e) {
               float v0 = o[c * 8 + 2 * e] * inv_l, v1 = o[c * 8 + 2 * e + 1] * inv_l;
               if (kGate) {
-                v0 *= 1.f / (1.f + __expf(-g[c * 8 + 2 * e]));
-                v1 *= 1.f / (1.f + __expf(-g[c * 8 + 2 * e + 1]));
+                v0 *= sigmoid_fast(g[c * 8 + 2 * e]);
+                v1 *= sigmoid_fast(g[c * 8 + 2 * e + 1]);
               }
               wv[e] = pack_bf16x2(v0, v1);
             }

@@ -334,6 +334,20 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// tanh on the MUFU unit (tanh.approx.f32, an approximation with an error of
+// order 2^-11).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation where 1 / (1 + e^-x)
+// needs an exponential and a reciprocal.  Its error (half that of the tanh)
+// lies far below the bf16 rounding of the gated output; the parity tests
+// compare the gated outputs with the oracle's fp64 sigmoid.
+__device__ __forceinline__ float sigmoid_fast(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
+
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -527,8 +527,8 @@ __global__ void __launch_bounds__(kPwaThreads, 1) pba_pwa_sm100_kernel(const __g
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const float o0 = __uint_as_float(r[8 * q + 2 * e]), o1 = __uint_as_float(r[8 * q + 2 * e + 1]);
-                ow[4 * q + e] = pack_bf16x2(o0 / (1.f + __expf(-bf16lo_to_f32(gw[e]))),
-                                            o1 / (1.f + __expf(-bf16hi_to_f32(gw[e]))));
+                ow[4 * q + e] = pack_bf16x2(o0 * sigmoid_fast(bf16lo_to_f32(gw[e])),
+                                            o1 * sigmoid_fast(bf16hi_to_f32(gw[e])));
               }
             }
           } else {
