@@ -86,7 +86,11 @@ typedef enum { PBA_TRI_STARTING = 0, PBA_TRI_ENDING = 1 } pba_tri_orient;
  *   B, H       batch and heads (B, H >= 1)
  *   Nq, Nk     query rows and keys (>= 0; Nk = 0 makes every row empty)
  *   D          head dimension: 32 or 64 (bf16 and fp32)
- *   dtype      pba_dtype of q, k, v, bias and of pba_forward's `out`
+ *   dtype      pba_dtype of q, k, v, bias and of pba_forward's `out`.  bf16
+ *              runs on the tensor cores; fp32 is the reference-precision
+ *              path (CUDA cores, one warp per query row, fp32 end to end,
+ *              about 1e-5 from the exact result): meant for checks and small
+ *              problems, orders of magnitude slower than bf16 at size.
  *   softmax_scale  tau; 0 selects 1/sqrt(D).  The bias is added unscaled.
  *   *_stride   strides in ELEMENTS of the (b, h, n) axes; the d axis (and
  *              the key axis of the bias) has stride 1.

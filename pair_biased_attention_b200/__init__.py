@@ -185,7 +185,9 @@ def pba_forward(q, k, v, bias, key_mask=None, out=None, lse=None, softmax_scale=
                 stream=None):
     """O (and the natural-log log-sum-exp) of pair-biased attention over all
     keys.  q [B,H,Nq,D], k/v [B,H,Nk,D], bias [B|1,H|1,Nq,Nk] (bf16 or fp32, all
-    the same dtype), key_mask [B,Nk] uint8 (1 = key takes part) or None."""
+    the same dtype), key_mask [B,Nk] uint8 (1 = key takes part) or None.
+    bf16 runs on the tensor cores; fp32 is the reference-precision path on the
+    CUDA cores (fp32 end to end), meant for checks and small problems."""
     for n, t in (("q", q), ("k", k), ("v", v), ("bias", bias)):
         _cuda(n, t, q.dtype)
     _cuda("key_mask", key_mask, torch.uint8)
