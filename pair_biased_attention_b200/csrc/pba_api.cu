@@ -14,6 +14,7 @@
 
 #include "pba.h"
 #include "pba_attn_sm100.cuh"
+#include "pba_attn_tf32_sm100.cuh"
 #include "pba_proj_sm100.cuh"
 #include "pba_oproj_sm100.cuh"
 #include "pba_pwa_sm100.cuh"
@@ -88,16 +89,16 @@ cudaError_t once_per_device(PerDeviceOnce &o, F &&setup) {
 
 constexpr int64_t kMaxI32 = 2147483647;
 
-// 4-D tiled tensor map of bf16 elements.  dims/strides innermost first;
-// strides in bytes for dims 1..3.  A dim of extent 1 gets a harmless positive
-// stride (its coordinate is always 0).
+// 4-D tiled tensor map of bf16 (or, with f32, fp32) elements.  dims/strides
+// innermost first; strides in bytes for dims 1..3.  A dim of extent 1 gets a
+// harmless positive stride (its coordinate is always 0).
 bool make_map(CUtensorMap *map, const void *base, const uint64_t dims[4], const int64_t strides_bytes[3],
-              const uint32_t box[4], CUtensorMapSwizzle swizzle) {
+              const uint32_t box[4], CUtensorMapSwizzle swizzle, bool f32 = false) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t gdim[4] = {dims[0], dims[1], dims[2], dims[3]};
   cuuint64_t gstride[3];
-  int64_t prev_extent = int64_t(dims[0]) * 2;
+  int64_t prev_extent = int64_t(dims[0]) * (f32 ? 4 : 2);
   for (int i = 0; i < 3; ++i) {
     int64_t s = strides_bytes[i];
     if (dims[i + 1] == 1 || s <= 0) s = (prev_extent + 15) / 16 * 16;
@@ -106,13 +107,14 @@ bool make_map(CUtensorMap *map, const void *base, const uint64_t dims[4], const 
   }
   cuuint32_t bdim[4] = {box[0], box[1], box[2], box[3]};
   cuuint32_t estride[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), gdim, gstride, bdim, estride,
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), gdim, gstride, bdim, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 bool stride_ok_bf16(int64_t s, int64_t extent) { return extent <= 1 || (s > 0 && s % 8 == 0); }
+bool stride_ok_f32(int64_t s, int64_t extent) { return extent <= 1 || (s > 0 && s % 4 == 0); }
 
 // ------------------------------------------------------------ tensor-core path
 struct TcProblem {
@@ -254,6 +256,102 @@ pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
   return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------ fp32 on the tensor cores
+template <int D, bool kPartial, bool kMasked>
+cudaError_t launch_tf32(const pba::Tf32Params &p, int64_t grid, cudaStream_t stream) {
+  using L = pba::Tf32Layout<D>;
+  auto kern = pba::pba_attn_tf32_sm100_kernel<D, kPartial, kMasked>;
+  static PerDeviceOnce once;
+  const cudaError_t attr_err = once_per_device(
+      once, [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc); });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<unsigned(grid), pba::kTfThreads, L::kSmemAlloc, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_tf32(const pba::Tf32Params &p, int64_t grid, bool partial, bool masked, cudaStream_t st) {
+  if (partial) return masked ? launch_tf32<D, true, true>(p, grid, st) : launch_tf32<D, true, false>(p, grid, st);
+  return masked ? launch_tf32<D, false, true>(p, grid, st) : launch_tf32<D, false, false>(p, grid, st);
+}
+
+// fp32 inputs whose tiles the Tensor Memory Accelerator can load (16-byte
+// aligned bases and row strides) run on the tensor cores; the caller routes
+// the others to the CUDA-core kernel.
+bool tf32_layout_ok(const pba_attn_desc *d, const void *q, const void *k, const void *v, const void *bias,
+                    const void *out) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) || !aligned16(out)) return false;
+  const int64_t *qs = d->q_stride, *ks = d->k_stride, *vs = d->v_stride, *bs = d->bias_stride, *os = d->out_stride;
+  if (!stride_ok_f32(qs[0], d->B) || !stride_ok_f32(qs[1], d->H) || !stride_ok_f32(qs[2], d->Nq) ||
+      !stride_ok_f32(ks[0], d->B) || !stride_ok_f32(ks[1], d->H) || !stride_ok_f32(ks[2], d->Nk) ||
+      !stride_ok_f32(vs[0], d->B) || !stride_ok_f32(vs[1], d->H) || !stride_ok_f32(vs[2], d->Nk) ||
+      !stride_ok_f32(bs[2], d->Nq))
+    return false;
+  if ((bs[0] != 0 && !stride_ok_f32(bs[0], d->B)) || (bs[1] != 0 && !stride_ok_f32(bs[1], d->H))) return false;
+  for (int i = 0; i < 3; ++i)
+    if (os[i] % 4 != 0) return false;  // 16-byte stores of whole output rows
+  return true;
+}
+
+pba_status run_tf32(const pba_attn_desc *d, float tau, const void *q, const void *k, const void *v, const void *bias,
+                    const uint8_t *mask, bool partial, void *out, float *lse, float *l_part, cudaStream_t stream) {
+  pba::Tf32Params p;
+  std::memset(&p, 0, sizeof(p));
+  const int64_t B = d->B, H = d->H, Nq = d->Nq, Nk = d->Nk, D = d->D;
+  const int64_t *qs = d->q_stride, *ks = d->k_stride, *vs = d->v_stride, *bs = d->bias_stride;
+  {
+    // Q, K, V [B][H][n][D] as (D, n, H, B): 32-feature boxes of 128 query / 64 key rows
+    const uint64_t dq[4] = {uint64_t(D), uint64_t(Nq), uint64_t(H), uint64_t(B)};
+    const uint64_t dk[4] = {uint64_t(D), uint64_t(Nk), uint64_t(H), uint64_t(B)};
+    const int64_t sq[3] = {qs[2] * 4, qs[1] * 4, qs[0] * 4};
+    const int64_t sk[3] = {ks[2] * 4, ks[1] * 4, ks[0] * 4};
+    const int64_t sv[3] = {vs[2] * 4, vs[1] * 4, vs[0] * 4};
+    const uint32_t qbox[4] = {32, uint32_t(pba::kTfBM), 1, 1};
+    const uint32_t kbox[4] = {32, uint32_t(pba::kTfBN), 1, 1};
+    if (!make_map(&p.tm_q, q, dq, sq, qbox, CU_TENSOR_MAP_SWIZZLE_128B, true) ||
+        !make_map(&p.tm_k, k, dk, sk, kbox, CU_TENSOR_MAP_SWIZZLE_128B, true) ||
+        !make_map(&p.tm_v, v, dk, sv, kbox, CU_TENSOR_MAP_SWIZZLE_128B, true))
+      return PBA_ERR_INVALID_ARG;
+  }
+  {
+    // bias [B|1][H|1][Nq][Nk] as (keys, rows, H, B): 32-key boxes of 128 rows
+    const uint64_t hb = bs[1] == 0 ? 1 : uint64_t(H), bb = bs[0] == 0 ? 1 : uint64_t(B);
+    const uint64_t dims[4] = {uint64_t(Nk), uint64_t(Nq), hb, bb};
+    const int64_t st[3] = {bs[2] * 4, bs[1] * 4, bs[0] * 4};
+    const uint32_t box[4] = {32, uint32_t(pba::kTfBM), 1, 1};
+    if (!make_map(&p.tm_bias, bias, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B, true)) return PBA_ERR_INVALID_ARG;
+  }
+  p.B = int(B);
+  p.H = int(H);
+  p.Nq = int(Nq);
+  p.Nk = int(Nk);
+  p.n_qblocks = int((Nq + pba::kTfBM - 1) / pba::kTfBM);
+  const int64_t grid = B * H * p.n_qblocks;
+  if (grid > kMaxI32) return PBA_ERR_INVALID_ARG;
+  p.bias_h_bcast = bs[1] == 0;
+  p.bias_b_bcast = bs[0] == 0;
+  p.mask = mask;
+  p.mask_sb = d->mask_stride_b;
+  p.mask_vec16 = mask != nullptr && aligned16(mask) && (B == 1 || d->mask_stride_b % 16 == 0);
+  p.tau = tau;
+  p.out = static_cast<float *>(out);
+  p.out_sb = d->out_stride[0];
+  p.out_sh = d->out_stride[1];
+  p.out_sn = d->out_stride[2];
+  p.lse = lse;
+  p.lse_sb = d->lse_stride[0];
+  p.lse_sh = d->lse_stride[1];
+  p.lse_sn = d->lse_stride[2];
+  p.l_part = l_part;
+  p.err = device_error_word();
+  if (p.err == nullptr) return PBA_ERR_CUDA;
+  p.timeout_ns = g_timeout_ns.load();
+  const bool masked = mask != nullptr || Nk % pba::kTfBN != 0;
+  const cudaError_t e = (D == 64) ? dispatch_tf32<64>(p, grid, partial, masked, stream)
+                                  : dispatch_tf32<32>(p, grid, partial, masked, stream);
+  return e == cudaSuccess ? PBA_OK : PBA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------ shared checks
 pba_status check_desc(const pba_attn_desc *d) {
   if (d == nullptr) return PBA_ERR_INVALID_ARG;
@@ -306,7 +404,10 @@ pba_status attn_common(const pba_attn_desc *d, const void *q, const void *k, con
   if (d->Nk == 0) return launch_empty(d, partial, out, lse, l_part, stream);
   const float tau = tau_of(d->softmax_scale, d->D);
 
+  if (d->dtype == PBA_F32 && tf32_layout_ok(d, q, k, v, bias, out))
+    return run_tf32(d, tau, q, k, v, bias, mask, partial, out, lse, l_part, stream);
   if (d->dtype == PBA_F32) {
+    // rows the tile loads cannot address: one warp per query row on the CUDA cores
     pba::SimtParams p;
     p.B = int(d->B);
     p.H = int(d->H);
