@@ -328,7 +328,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "oproj1024", "pwa4k", "bwd4k",
+    ap.add_argument("--profile", choices=["none", "pba4k", "tri512", "proj1024", "oproj1024", "pwa4k", "bwd4k", "f32_4k",
                                           "merge8k"],
                     default="none",
                     help="run one small case only (for ncu captures); prints no JSON line")
@@ -427,6 +427,7 @@ def main():
     line["pwa"] = run_pwa(args, pba, dev, stream, pg, peaks, clk)
     line["backward"] = run_bwd(args, pba, dev, stream, pg, peaks)
     line["ring8k"] = run_ring8k(args, pba, dev, stream, pg, peaks)
+    line["f32"] = run_f32(args, pba, dev, stream, pg, peaks)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -588,6 +589,57 @@ def run_bwd(args, pba, dev, stream, pg, peaks):
                          "tensor_frac": (flops / (ms / 1e3) / 1e12) / peaks["bf16_tflops"]}}
 
 
+# Nominal dense tf32 : bf16 tensor rate of the B200 (1.1 : 2.25 PFLOP/s): the
+# tf32 peak is the measured bf16 peak times this ratio.
+TF32_PER_BF16 = 1.1 / 2.25
+
+
+def run_f32(args, pba, dev, stream, pg, peaks):
+    """pba_forward with fp32 inputs on the ring8k shapes (N=8192, H=16, D=64,
+    bias ~N(0,1), no mask), timed on its own after the step: K calls after 3
+    warm-up calls, CUDA events on the stream; plus the pr1 config (fp32, N=256,
+    H=4, D=32), which is a single wave of 8 CTAs and measures launch latency
+    more than throughput.  The path runs three tf32 products per product
+    (high and low parts of both operands), so its tensor-core work is three
+    times the algorithmic 4*H*N^2*D FLOPs; that work is reported against the
+    tf32 peak (the measured bf16 peak times the nominal tf32 : bf16 ratio)."""
+    cfg = W.RING8K
+    q, k, v, bias = (t.float() for t in W.attn_inputs(cfg, dev)[:4])
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+
+    def timed(call, n):
+        for _ in range(3):
+            call()
+        barrier(pg)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(n):
+            call()
+        e.record(stream)
+        barrier(pg)
+        return max_over_ranks(s.elapsed_time(e), pg) / n
+
+    ms = timed(lambda: pba.pba_forward(q, k, v, bias, None, out, lse, stream=stream), args.steps)
+    del q, k, v, bias, out, lse
+    pq, pk, pv, pb, _ = W.attn_inputs(W.PR1, dev)
+    pout = torch.empty_like(pq)
+    plse = torch.empty(pq.shape[:3], dtype=torch.float32, device=dev)
+    pr1_ms = timed(lambda: pba.pba_forward(pq, pk, pv, pb, None, pout, plse, stream=stream), args.steps)
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("the fp32 attention kernel recorded a device error")
+    flops = attn_flops(cfg.B, cfg.H, cfg.N, cfg.N, cfg.D)
+    alg = flops / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"] * TF32_PER_BF16
+    return {"ms_per_call": ms, "calls": args.steps, "gpu_launches": args.steps, "tflops_algorithmic": alg,
+            "workload": f"ring8k shapes in fp32: N={cfg.N} H={cfg.H} D={cfg.D}, bias ~N(0,1), no mask",
+            "pr1_ms_per_call": pr1_ms,
+            "roofline": {"bound": "tensor", "achieved": 3 * alg, "peak": peak, "unit": "TFLOP/s",
+                         "frac": 3 * alg / peak, "kernel": "pba_attn_tf32_sm100_kernel (pba_forward, fp32)",
+                         "peak_source": peaks["source"] + " bf16 x 1.1/2.25",
+                         "note": "achieved = tf32 tensor-core work, 3x the algorithmic FLOPs"}}
+
+
 def merge_bytes(P, rows, D, out_elt=2):
     """Algorithmic bytes of softmax_merge: the P partials (O_p fp32, m_p, l_p)
     read once, out and lse written once."""
@@ -716,7 +768,8 @@ def run_profile_case(args, pba, dev):
     than L2); merge8k = softmax_merge of the ring8k partials (L2 flushed
     before each merge); tri512 = triangle attention N=512 both orientations; proj1024 /
     oproj1024 = the input / output projections at tri1024; pwa4k = pwa_forward;
-    bwd4k = pba_backward at N=4096, H=4."""
+    bwd4k = pba_backward at N=4096, H=4; f32_4k = pba_forward with fp32 inputs
+    at N=4096, H=16, D=64 (bias 1 GB)."""
     if args.profile == "merge8k":
         cfg = W.RING8K
         q, k, v, bias, _ = W.attn_inputs(cfg, dev)
@@ -753,6 +806,10 @@ def run_profile_case(args, pba, dev):
         w_o = (torch.randn((cfg.H * cfg.D, cfg.c), generator=g, device=dev) / (cfg.H * cfg.D) ** 0.5).to(torch.bfloat16)
         for _ in range(2):
             pba.tri_out_proj_forward(o, w_o)
+    elif args.profile == "f32_4k":
+        q, k, v, bias, _ = W.random_attn(1, 16, 4096, 4096, 64, dtype=torch.float32, seed=1, device=dev)
+        for _ in range(2):
+            pba.pba_forward(q, k, v, bias)
     elif args.profile == "pba4k":
         cfg = W.AttnConfig("pba4k", B=1, N=4096, H=16, D=64, dtype=torch.bfloat16, seed=4, mask="random5")
         q, k, v, bias, mask = W.attn_inputs(cfg, dev)

@@ -262,8 +262,15 @@ cudaError_t launch_tf32(const pba::Tf32Params &p, int64_t grid, cudaStream_t str
   using L = pba::Tf32Layout<D>;
   auto kern = pba::pba_attn_tf32_sm100_kernel<D, kPartial, kMasked>;
   static PerDeviceOnce once;
-  const cudaError_t attr_err = once_per_device(
-      once, [&] { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc); });
+  const cudaError_t attr_err = once_per_device(once, [&] {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemAlloc);
+    // the warpgroup register split must fit in what the block is launched with
+    cudaFuncAttributes fa;
+    if (e == cudaSuccess && cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+        fa.numRegs * pba::kTfThreads < pba::kTfRegSplitTotal)
+      e = cudaErrorInvalidConfiguration;
+    return e;
+  });
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<unsigned(grid), pba::kTfThreads, L::kSmemAlloc, stream>>>(p);
   return cudaGetLastError();

@@ -19,28 +19,34 @@
 // 3 * 2^-22 |x y| per product (the split of "Recovering single precision
 // accuracy from Tensor Cores while surpassing the FP32 theoretical peak
 // performance", Ootomo and Yokota, 2022).  The sums are the tensor core's
-// fp32 accumulation.  This applies to S = Q K^T (Q, K split in shared memory)
-// and to O += P V (P split by the softmax threads into Tensor Memory, V split
-// and transposed in shared memory).
+// fp32 accumulation.  This applies to S = Q K^T (Q's high part and K's two
+// parts in shared memory, Q's low part in Tensor Memory) and to O += P V (P
+// split by the softmax threads into Tensor Memory, V split and transposed in
+// shared memory).
 //
 // Operand layouts: every operand is K-major (the contraction dimension
-// contiguous) with the 128-byte swizzle: Q and K rows are D fp32 (one or two
-// 128-byte chunks of 32 elements), P is read from Tensor Memory, and V, which
-// arrives key-major, is written transposed (one row per feature, keys
-// contiguous) by the split warps.
+// contiguous).  Q's two parts and P's two parts are the A operands, read from
+// Tensor Memory; K's parts and V^T's parts are the B operands, in shared
+// memory with the 128-byte swizzle (rows of D or 64 fp32 as 128-byte chunks of
+// 32).  V arrives key-major and is written transposed (one row per feature,
+// keys contiguous) by its split warps.
 //
-// One CTA per (b, h, 128 query rows):
-//   warps 0-3   softmax (thread t owns query row t)
-//   warps 4-7   split: Q once, then per key tile K (in place + low part) and
-//               V (transposed high and low parts)
-//   warp 8      TMA producer of Q, K and V
-//   warp 9      allocates Tensor Memory and issues every tcgen05.mma
-//   warp 10     TMA producer of the bias tiles
+// One CTA per (b, h, 128 query rows), sixteen warps:
+//   warps 0-3    softmax (thread t owns query row t)
+//   warps 4-7    K split: Q once (row by row, both parts into Tensor Memory),
+//                then per key tile K (high part in place, low part beside it)
+//   warps 8-11   V split: per key tile V^T's high and low parts
+//   warp 12      TMA producer of Q, K and V
+//   warp 13      allocates Tensor Memory and issues every tcgen05.mma
+//   warp 14      TMA producer of the bias tiles
+//   warp 15      no role (completes the fourth warpgroup)
 // Tensor Memory (512 columns x 128 lanes of fp32):
-//   [0,64) S0  [64,128) S1  [128,192) P_hi0  [192,256) P_hi1
-//   [256,320) P_lo0  [320,384) P_lo1  [384,384+D) O
-// Issue order of the MMA warp: S(0), S(1), PV(0), S(2), PV(1), ...: the next
-// score tile is computed while the softmax works on the current one.
+//   [0,64) S0  [64,128) S1  [128,192) P_hi  [192,256) P_lo  [256,256+D) O
+//   [256+D,256+2D) Q_hi  [256+2D,256+3D) Q_lo
+// Issue order of the MMA warp: S(0), S(1), PV(0), S(2), PV(1), ...  The K and
+// V splits run on their own warps, ahead of the MMAs by their ring depths, so
+// the tensor pipe, not a chain of loads and splits, sets the pace: a tile is
+// S(j+1) and PV(j) back to back, while the softmax works on tile j+1.
 #pragma once
 
 #include <cuda.h>
@@ -51,13 +57,18 @@ namespace pba {
 
 constexpr int kTfBM = 128;  // query rows per CTA (one TMEM lane each)
 constexpr int kTfBN = 64;   // keys per tile
-constexpr int kTfThreads = 352;
-constexpr int kTfWarpSplit0 = 4;
-constexpr int kTfWarpProducer = 8;
-constexpr int kTfWarpMma = 9;
-constexpr int kTfWarpBias = 10;
+constexpr int kTfThreads = 512;
+constexpr int kTfWarpKSplit0 = 4;
+constexpr int kTfWarpVSplit0 = 8;
+constexpr int kTfWarpProducer = 12;
+constexpr int kTfWarpMma = 13;
+constexpr int kTfWarpBias = 14;
 constexpr uint32_t kTfTmemCols = 512;
-constexpr uint32_t kTfColS = 0, kTfColPhi = 128, kTfColPlo = 256, kTfColO = 384;
+constexpr uint32_t kTfColS = 0, kTfColPhi = 128, kTfColPlo = 192, kTfColO = 256;
+// Per-thread register limits after the warpgroup reallocation (launch: 128).
+constexpr int kTfRegsSoftmax = 248;
+constexpr int kTfRegsOther = 88;
+constexpr int kTfRegSplitTotal = 128 * kTfRegsSoftmax + 384 * kTfRegsOther;
 
 struct Tf32Params {
   CUtensorMap tm_q, tm_k, tm_v, tm_bias;
@@ -90,19 +101,23 @@ struct Tf32Layout {
   static constexpr int kVtBytes = 2 * kVtChunkBytes;    // 64 keys
   static constexpr int kBiasBoxBytes = kTfBM * 128;     // 128 rows x 32 keys
   static constexpr int kBiasBytes = 2 * kBiasBoxBytes;  // 64 keys
-  static constexpr int kKStages = (D == 32) ? 2 : 1;
-  static constexpr int kVRawStages = (D == 32) ? 2 : 1;
-  static constexpr int kVtStages = (D == 32) ? 2 : 1;
+  static constexpr int kKStages = (D == 32) ? 3 : 2;
+  static constexpr int kVRawStages = (D == 32) ? 3 : 2;
+  static constexpr int kVtStages = (D == 32) ? 3 : 2;
   static constexpr int kBiasStages = 2;
-  static constexpr int kOffQhi = 0;
-  static constexpr int kOffQlo = kOffQhi + kQBytes;
-  static constexpr int kOffKhi = kOffQlo + kQBytes;
+  static constexpr uint32_t kColQhi = kTfColO + D;
+  static constexpr uint32_t kColQlo = kTfColO + 2 * D;
+  static constexpr int kOffKhi = 0;
   static constexpr int kOffKlo = kOffKhi + kKStages * kKBytes;
   static constexpr int kOffVraw = kOffKlo + kKStages * kKBytes;
   static constexpr int kOffVthi = kOffVraw + kVRawStages * kKBytes;
   static constexpr int kOffVtlo = kOffVthi + kVtStages * kVtBytes;
   static constexpr int kOffBias = kOffVtlo + kVtStages * kVtBytes;
   static constexpr int kOffBar = kOffBias + kBiasStages * kBiasBytes;
+  // Q lands in the V^T high-part ring, which its split empties before the
+  // V split writes the first V^T tile there
+  static constexpr int kOffQraw = kOffVthi;
+  static_assert(kVtStages * kVtBytes >= kQBytes, "Q staging");
   // barriers
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQReady = 1;
@@ -116,17 +131,19 @@ struct Tf32Layout {
   static constexpr int kBarBiasFull = kBarVtEmpty + kVtStages;
   static constexpr int kBarBiasEmpty = kBarBiasFull + kBiasStages;
   static constexpr int kBarSFull = kBarBiasEmpty + kBiasStages;  // [2]
-  static constexpr int kBarSFree = kBarSFull + 2;
+  static constexpr int kBarSFree = kBarSFull + 2;                // [2]
   static constexpr int kBarPFull = kBarSFree + 2;
-  static constexpr int kBarPFree = kBarPFull + 2;  // [2]: P V of that buffer done
-  static constexpr int kBarDrain = kBarPFree + 2;
+  static constexpr int kBarPDone = kBarPFull + 1;  // a P V has completed
+  static constexpr int kBarDrain = kBarPDone + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemSlot + 4;
   static constexpr int kBytes = kOffAbort + 4;
   static constexpr int kSmemAlloc = kBytes + 1024;  // room to align the base to 1024
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
-  static_assert(kOffKhi % 1024 == 0 && kOffVthi % 1024 == 0 && kOffBias % 1024 == 0, "swizzle atoms");
+  static_assert(kOffKlo % 1024 == 0 && kOffVraw % 1024 == 0 && kOffVthi % 1024 == 0 && kOffVtlo % 1024 == 0 &&
+                    kOffBias % 1024 == 0,
+                "swizzle atoms");
 };
 
 // Splits four fp32 values into their tf32 high parts and tf32 low parts.
@@ -141,16 +158,23 @@ __device__ __forceinline__ void tf32_split4(const uint4 v, uint4 &hi, uint4 &lo)
   lo.w = to_tf32(__uint_as_float(v.w) - __uint_as_float(hi.w));
 }
 
-// Splits `bytes` of fp32 at `hi` in place and writes the low parts at the same
-// offsets from `lo` (the split is element-wise, so any swizzle carries over).
-// Thread st of the 128 split threads takes 16-byte words st, st + 128, ...
-__device__ __forceinline__ void tf32_split_tile(uint8_t *hi, uint8_t *lo, int bytes, int st) {
-  for (int off = st * 16; off < bytes; off += 128 * 16) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(hi + off);
+// Splits kBytes of fp32 at `hi` in place and writes the low parts at the
+// same offsets from `lo` (the split is element-wise, so any swizzle carries
+// over).  Thread st of 128 takes 16-byte words st, st + 128, ...; all loads
+// are issued before the first store.
+template <int kBytes>
+__device__ __forceinline__ void tf32_split_tile(uint8_t *hi, uint8_t *lo, int st) {
+  constexpr int kWords = kBytes / (128 * 16);
+  static_assert(kBytes % (128 * 16) == 0, "whole words per thread");
+  uint4 v[kWords];
+#pragma unroll
+  for (int i = 0; i < kWords; ++i) v[i] = *reinterpret_cast<const uint4 *>(hi + (i * 128 + st) * 16);
+#pragma unroll
+  for (int i = 0; i < kWords; ++i) {
     uint4 h, l;
-    tf32_split4(v, h, l);
-    *reinterpret_cast<uint4 *>(hi + off) = h;
-    *reinterpret_cast<uint4 *>(lo + off) = l;
+    tf32_split4(v[i], h, l);
+    *reinterpret_cast<uint4 *>(hi + (i * 128 + st) * 16) = h;
+    *reinterpret_cast<uint4 *>(lo + (i * 128 + st) * 16) = l;
   }
 }
 
@@ -238,9 +262,9 @@ __global__ void __launch_bounds__(kTfThreads, 1) pba_attn_tf32_sm100_kernel(cons
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[L::kBarSFull + i], 1);
       mbar_init(&bars[L::kBarSFree + i], kTfBM);
-      mbar_init(&bars[L::kBarPFull + i], kTfBM);
-      mbar_init(&bars[L::kBarPFree + i], 1);
     }
+    mbar_init(&bars[L::kBarPFull], kTfBM);
+    mbar_init(&bars[L::kBarPDone], 1);
     mbar_init(&bars[L::kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -264,173 +288,206 @@ __global__ void __launch_bounds__(kTfThreads, 1) pba_attn_tf32_sm100_kernel(cons
   int drain_abort = 0;
   wc_drain.abort_flag = &drain_abort;
 
-  if (warp == kTfWarpProducer) {
-    // ================================================================ Q/K/V TMA producer
-    if (lane == 0) {
-      const uint64_t pol_stream = l2_policy_evict_first();
-      const uint64_t pol_keep = l2_policy_evict_last();
-      bool ok = true;
-      int nk = 0, nv = 0;  // K and V tiles issued
-      mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
-#pragma unroll
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_4d(smem + L::kOffQhi + c * L::kQChunkBytes, &p.tm_q, &bars[L::kBarQFull], c * 32, q0, h, b,
-                    pol_stream);
-      for (int j = 0; j < nt && ok; ++j) {
-        const int sk = j % L::kKStages;
-        if (j >= L::kKStages && !(ok = mbar_wait(&bars[L::kBarKEmpty + sk], ((j / L::kKStages) - 1) & 1, wc)))
-          break;
-        mbar_arrive_expect_tx(&bars[L::kBarKFull + sk], L::kKBytes);
-#pragma unroll
+  // Registers: the launch gives 128 per thread (512 x 128 = 65536); the
+  // split, producer and MMA warpgroups give part of theirs to the softmax
+  // warpgroup (128 x 248 + 384 x 88 = 65536).  Each warpgroup changes its
+  // limit once, at the top of its own branch.
+  if (warp >= kTfWarpProducer) {
+    setmaxnreg_dec<kTfRegsOther>();
+    if (warp == kTfWarpProducer) {
+      // ================================================================ Q/K/V TMA producer
+      if (lane == 0) {
+        const uint64_t pol_stream = l2_policy_evict_first();
+        const uint64_t pol_keep = l2_policy_evict_last();
+        bool ok = true;
+        int nk = 0, nv = 0;  // K and V tiles issued
+        mbar_arrive_expect_tx(&bars[L::kBarQFull], L::kQBytes);
+  #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kOffKhi + sk * L::kKBytes + c * L::kKChunkBytes, &p.tm_k, &bars[L::kBarKFull + sk],
-                      c * 32, j * kTfBN, h, b, pol_keep);
-        ++nk;
-        const int sv = j % L::kVRawStages;
-        if (j >= L::kVRawStages &&
-            !(ok = mbar_wait(&bars[L::kBarVRawEmpty + sv], ((j / L::kVRawStages) - 1) & 1, wc)))
-          break;
-        mbar_arrive_expect_tx(&bars[L::kBarVFull + sv], L::kKBytes);
-#pragma unroll
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_load_4d(smem + L::kOffVraw + sv * L::kKBytes + c * L::kKChunkBytes, &p.tm_v, &bars[L::kBarVFull + sv],
-                      c * 32, j * kTfBN, h, b, pol_keep);
-        ++nv;
-      }
-      if (!ok) {
-        // Let every copy already issued land before the CTA exits: slot s of a
-        // ring of S slots was armed (n - s + S - 1) / S times after n issues.
-        mbar_wait(&bars[L::kBarQFull], 0, wc_drain);
-        for (int s = 0; s < L::kKStages; ++s) {
-          const int a = (nk - s + L::kKStages - 1) / L::kKStages;
-          if (a > 0) mbar_wait(&bars[L::kBarKFull + s], (a - 1) & 1, wc_drain);
+          tma_load_4d(smem + L::kOffQraw + c * L::kQChunkBytes, &p.tm_q, &bars[L::kBarQFull], c * 32, q0, h, b,
+                      pol_stream);
+        for (int j = 0; j < nt && ok; ++j) {
+          const int sk = j % L::kKStages;
+          if (j >= L::kKStages && !(ok = mbar_wait(&bars[L::kBarKEmpty + sk], ((j / L::kKStages) - 1) & 1, wc)))
+            break;
+          mbar_arrive_expect_tx(&bars[L::kBarKFull + sk], L::kKBytes);
+  #pragma unroll
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(smem + L::kOffKhi + sk * L::kKBytes + c * L::kKChunkBytes, &p.tm_k, &bars[L::kBarKFull + sk],
+                        c * 32, j * kTfBN, h, b, pol_keep);
+          ++nk;
+          const int sv = j % L::kVRawStages;
+          if (j >= L::kVRawStages &&
+              !(ok = mbar_wait(&bars[L::kBarVRawEmpty + sv], ((j / L::kVRawStages) - 1) & 1, wc)))
+            break;
+          mbar_arrive_expect_tx(&bars[L::kBarVFull + sv], L::kKBytes);
+  #pragma unroll
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_4d(smem + L::kOffVraw + sv * L::kKBytes + c * L::kKChunkBytes, &p.tm_v, &bars[L::kBarVFull + sv],
+                        c * 32, j * kTfBN, h, b, pol_keep);
+          ++nv;
         }
-        for (int s = 0; s < L::kVRawStages; ++s) {
-          const int a = (nv - s + L::kVRawStages - 1) / L::kVRawStages;
-          if (a > 0) mbar_wait(&bars[L::kBarVFull + s], (a - 1) & 1, wc_drain);
-        }
-      }
-    }
-  } else if (warp == kTfWarpBias) {
-    // ================================================================ bias TMA producer
-    if (lane == 0) {
-      const uint64_t pol_stream = l2_policy_evict_first();
-      const int hb = p.bias_h_bcast ? 0 : h;
-      const int bb = p.bias_b_bcast ? 0 : b;
-      bool ok = true;
-      int nb = 0;
-      for (int j = 0; j < nt && ok; ++j) {
-        const int s = j % L::kBiasStages;
-        if (j >= L::kBiasStages &&
-            !(ok = mbar_wait(&bars[L::kBarBiasEmpty + s], ((j / L::kBiasStages) - 1) & 1, wc)))
-          break;
-        mbar_arrive_expect_tx(&bars[L::kBarBiasFull + s], L::kBiasBytes);
-        // [128 queries][64 keys] as two 32-key boxes, 128-byte swizzle
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          tma_load_4d(smem + L::kOffBias + s * L::kBiasBytes + c * L::kBiasBoxBytes, &p.tm_bias,
-                      &bars[L::kBarBiasFull + s], j * kTfBN + c * 32, q0, hb, bb, pol_stream);
-        ++nb;
-      }
-      if (!ok)
-        for (int s = 0; s < L::kBiasStages; ++s) {
-          const int a = (nb - s + L::kBiasStages - 1) / L::kBiasStages;
-          if (a > 0) mbar_wait(&bars[L::kBarBiasFull + s], (a - 1) & 1, wc_drain);
-        }
-    }
-  } else if (warp == kTfWarpMma) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_tf32_f32(kTfBM, kTfBN);
-      const uint32_t idesc_o = idesc_tf32_f32(kTfBM, D);
-      constexpr uint32_t kDescHi = smem_desc_hi(1024, 2);  // 8-row atoms of 128 bytes, 128-byte swizzle
-      const uint32_t qhi = smem_desc_lo(smem_u32(smem + L::kOffQhi), 16);
-      const uint32_t qlo = smem_desc_lo(smem_u32(smem + L::kOffQlo), 16);
-      // S(buf) = Q K^T over D / 8 steps of 8 features, three products per step
-      // (low x high, high x low, high x high); a step's operands start 32 bytes
-      // further along a 128-byte swizzle row, or at the next 32-feature chunk.
-      auto issue_s = [&](int buf, int sk) {
-        const uint32_t d_tmem = tmem + kTfColS + buf * kTfBN;
-        const uint32_t khi = smem_desc_lo(smem_u32(smem + L::kOffKhi + sk * L::kKBytes), 16);
-        const uint32_t klo = smem_desc_lo(smem_u32(smem + L::kOffKlo + sk * L::kKBytes), 16);
-#pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t a = pass == 0 ? qlo : qhi, bk = pass == 1 ? klo : khi;
-#pragma unroll
-          for (int k = 0; k < D / 8; ++k) {
-            const uint32_t qa = uint32_t((k >> 2) * L::kQChunkBytes + (k & 3) * 32) >> 4;
-            const uint32_t ka = uint32_t((k >> 2) * L::kKChunkBytes + (k & 3) * 32) >> 4;
-            mma_tf32_ss(d_tmem, desc_at(a, qa, kDescHi), desc_at(bk, ka, kDescHi), idesc_s,
-                        (pass > 0 || k > 0) ? 1u : 0u);
+        if (!ok) {
+          // Let every copy already issued land before the CTA exits: slot s of a
+          // ring of S slots was armed (n - s + S - 1) / S times after n issues.
+          mbar_wait(&bars[L::kBarQFull], 0, wc_drain);
+          for (int s = 0; s < L::kKStages; ++s) {
+            const int a = (nk - s + L::kKStages - 1) / L::kKStages;
+            if (a > 0) mbar_wait(&bars[L::kBarKFull + s], (a - 1) & 1, wc_drain);
+          }
+          for (int s = 0; s < L::kVRawStages; ++s) {
+            const int a = (nv - s + L::kVRawStages - 1) / L::kVRawStages;
+            if (a > 0) mbar_wait(&bars[L::kBarVFull + s], (a - 1) & 1, wc_drain);
           }
         }
-        tc_commit(&bars[L::kBarSFull + buf]);
-      };
-      // O += P(buf) V over 8 steps of 8 keys: P from Tensor Memory (8 columns
-      // per step), V^T from shared memory (32 bytes per step inside a key chunk)
-      auto issue_pv = [&](int buf, int sv, bool first) {
-        const uint32_t d_tmem = tmem + kTfColO;
-        const uint32_t phi = tmem + kTfColPhi + buf * kTfBN, plo = tmem + kTfColPlo + buf * kTfBN;
-        const uint32_t vhi = smem_desc_lo(smem_u32(smem + L::kOffVthi + sv * L::kVtBytes), 16);
-        const uint32_t vlo = smem_desc_lo(smem_u32(smem + L::kOffVtlo + sv * L::kVtBytes), 16);
-#pragma unroll
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t a = pass == 0 ? plo : phi, bv = pass == 1 ? vlo : vhi;
-#pragma unroll
-          for (int k = 0; k < kTfBN / 8; ++k) {
-            const uint32_t va = uint32_t((k >> 2) * L::kVtChunkBytes + (k & 3) * 32) >> 4;
-            mma_tf32_ts(d_tmem, a + k * 8, desc_at(bv, va, kDescHi), idesc_o,
-                        (!first || pass > 0 || k > 0) ? 1u : 0u);
-          }
-        }
-        tc_commit(&bars[L::kBarPFree + buf]);
-      };
-      bool ok = mbar_wait(&bars[L::kBarQReady], 0, wc);
-      if (ok) ok = mbar_wait(&bars[L::kBarKReady], 0, wc);
-      if (ok) {
-        tc_fence_after_sync();
-        issue_s(0, 0);
-        tc_commit(&bars[L::kBarKEmpty]);
       }
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt) {
-          // S(j+1) into the other buffer: its K tile split, and S(j-1) read by the softmax
-          const int jn = j + 1, sk = jn % L::kKStages, buf = jn & 1;
-          ok = mbar_wait(&bars[L::kBarKReady + sk], (jn / L::kKStages) & 1, wc);
-          if (ok && jn >= 2) ok = mbar_wait(&bars[L::kBarSFree + buf], ((jn >> 1) - 1) & 1, wc);
+    } else if (warp == kTfWarpBias) {
+      // ================================================================ bias TMA producer
+      if (lane == 0) {
+        const uint64_t pol_stream = l2_policy_evict_first();
+        const int hb = p.bias_h_bcast ? 0 : h;
+        const int bb = p.bias_b_bcast ? 0 : b;
+        bool ok = true;
+        int nb = 0;
+        for (int j = 0; j < nt && ok; ++j) {
+          const int s = j % L::kBiasStages;
+          if (j >= L::kBiasStages &&
+              !(ok = mbar_wait(&bars[L::kBarBiasEmpty + s], ((j / L::kBiasStages) - 1) & 1, wc)))
+            break;
+          mbar_arrive_expect_tx(&bars[L::kBarBiasFull + s], L::kBiasBytes);
+          // [128 queries][64 keys] as two 32-key boxes, 128-byte swizzle
+  #pragma unroll
+          for (int c = 0; c < 2; ++c)
+            tma_load_4d(smem + L::kOffBias + s * L::kBiasBytes + c * L::kBiasBoxBytes, &p.tm_bias,
+                        &bars[L::kBarBiasFull + s], j * kTfBN + c * 32, q0, hb, bb, pol_stream);
+          ++nb;
+        }
+        if (!ok)
+          for (int s = 0; s < L::kBiasStages; ++s) {
+            const int a = (nb - s + L::kBiasStages - 1) / L::kBiasStages;
+            if (a > 0) mbar_wait(&bars[L::kBarBiasFull + s], (a - 1) & 1, wc_drain);
+          }
+      }
+    } else if (warp == kTfWarpMma) {
+      // ================================================================ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc_s = idesc_tf32_f32(kTfBM, kTfBN);
+        const uint32_t idesc_o = idesc_tf32_f32(kTfBM, D);
+        constexpr uint32_t kDescHi = smem_desc_hi(1024, 2);  // 8-row atoms of 128 bytes, 128-byte swizzle
+        // S(buf) = Q K^T over D / 8 steps of 8 features, three products per step
+        // (Q_lo x K_hi, Q_hi x K_lo, Q_hi x K_hi): Q from Tensor Memory (8
+        // columns per step), K from shared memory (32 bytes further along a
+        // 128-byte swizzle row per step, or the next 32-feature chunk).
+        auto issue_s = [&](int buf, int sk) {
+          const uint32_t d_tmem = tmem + kTfColS + buf * kTfBN;
+          const uint32_t khi = smem_desc_lo(smem_u32(smem + L::kOffKhi + sk * L::kKBytes), 16);
+          const uint32_t klo = smem_desc_lo(smem_u32(smem + L::kOffKlo + sk * L::kKBytes), 16);
+  #pragma unroll
+          for (int pass = 0; pass < 3; ++pass) {
+            const uint32_t a = tmem + (pass == 0 ? L::kColQlo : L::kColQhi);
+            const uint32_t bk = pass == 1 ? klo : khi;
+  #pragma unroll
+            for (int k = 0; k < D / 8; ++k) {
+              const uint32_t ka = uint32_t((k >> 2) * L::kKChunkBytes + (k & 3) * 32) >> 4;
+              mma_tf32_ts(d_tmem, a + k * 8, desc_at(bk, ka, kDescHi), idesc_s, (pass > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(&bars[L::kBarSFull + buf]);
+        };
+        // O += P V over 8 steps of 8 keys: P from Tensor Memory (8 columns per
+        // step), V^T from shared memory (32 bytes per step inside a key chunk).
+        auto issue_pv = [&](int sv, bool first) {
+          const uint32_t d_tmem = tmem + kTfColO;
+          const uint32_t vhi = smem_desc_lo(smem_u32(smem + L::kOffVthi + sv * L::kVtBytes), 16);
+          const uint32_t vlo = smem_desc_lo(smem_u32(smem + L::kOffVtlo + sv * L::kVtBytes), 16);
+  #pragma unroll
+          for (int pass = 0; pass < 3; ++pass) {
+            const uint32_t a = tmem + (pass == 0 ? kTfColPlo : kTfColPhi);
+            const uint32_t bv = pass == 1 ? vlo : vhi;
+  #pragma unroll
+            for (int k = 0; k < kTfBN / 8; ++k) {
+              const uint32_t va = uint32_t((k >> 2) * L::kVtChunkBytes + (k & 3) * 32) >> 4;
+              mma_tf32_ts(d_tmem, a + k * 8, desc_at(bv, va, kDescHi), idesc_o,
+                          (!first || pass > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          tc_commit(&bars[L::kBarPDone]);
+        };
+        bool ok = mbar_wait(&bars[L::kBarQReady], 0, wc);
+        if (ok) ok = mbar_wait(&bars[L::kBarKReady], 0, wc);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_s(0, 0);
+          tc_commit(&bars[L::kBarKEmpty]);
+        }
+        for (int j = 0; j < nt && ok; ++j) {
+          if (j + 1 < nt) {
+            // S(j+1) into the other buffer: its K tile split, and S(j-1) read by the softmax
+            const int jn = j + 1, sk = jn % L::kKStages, buf = jn & 1;
+            ok = mbar_wait(&bars[L::kBarKReady + sk], (jn / L::kKStages) & 1, wc);
+            if (ok && jn >= 2) ok = mbar_wait(&bars[L::kBarSFree + buf], ((jn >> 1) - 1) & 1, wc);
+            if (!ok) break;
+            tc_fence_after_sync();
+            issue_s(buf, sk);
+            tc_commit(&bars[L::kBarKEmpty + sk]);
+          }
+          // P V(j): V^T(j) split, P(j) written
+          const int sv = j % L::kVtStages;
+          ok = mbar_wait(&bars[L::kBarVtReady + sv], (j / L::kVtStages) & 1, wc);
+          if (ok) ok = mbar_wait(&bars[L::kBarPFull], j & 1, wc);
           if (!ok) break;
           tc_fence_after_sync();
-          issue_s(buf, sk);
-          tc_commit(&bars[L::kBarKEmpty + sk]);
+          issue_pv(sv, j == 0);
+          tc_commit(&bars[L::kBarVtEmpty + sv]);
         }
-        // P V(j): V^T(j) split, P(j) written
-        const int sv = j % L::kVtStages, buf = j & 1;
-        ok = mbar_wait(&bars[L::kBarVtReady + sv], (j / L::kVtStages) & 1, wc);
-        if (ok) ok = mbar_wait(&bars[L::kBarPFull + buf], (j >> 1) & 1, wc);
-        if (!ok) break;
-        tc_fence_after_sync();
-        issue_pv(buf, sv, j == 0);
-        tc_commit(&bars[L::kBarVtEmpty + sv]);
+        // Every MMA issued above completes before Tensor Memory is released.
+        tc_commit(&bars[L::kBarDrain]);
+        mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
       }
-      // Every MMA issued above completes before Tensor Memory is released.
-      tc_commit(&bars[L::kBarDrain]);
-      mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
     }
-  } else if (warp >= kTfWarpSplit0) {
-    // ================================================================ split warps
-    const int st = threadIdx.x - kTfWarpSplit0 * 32;
-    bool ok = mbar_wait(&bars[L::kBarQFull], 0, wc);
+    // warp 15 has no role
+  } else if (warp < kTfWarpVSplit0 && warp >= kTfWarpKSplit0) {
+    // ================================================================ K split warps
+    setmaxnreg_dec<kTfRegsOther>();
+    const int st = threadIdx.x - kTfWarpKSplit0 * 32;
+    // Q: thread st takes query row st, both parts into this warp's lanes of
+    // Tensor Memory
+    bool ok = warp_wait(&bars[L::kBarQFull], 0, wc);
     if (ok) {
-      tf32_split_tile(smem + L::kOffQhi, smem + L::kOffQlo, L::kQBytes, st);
-      fence_proxy_async_smem();
+      const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+      const uint8_t *qrow = smem + L::kOffQraw + st * 128;
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c) {
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(qrow + c * L::kQChunkBytes + ((g ^ (st & 7)) << 4));
+          uint4 h4, l4;
+          tf32_split4(v, h4, l4);
+          hi[4 * g] = h4.x, hi[4 * g + 1] = h4.y, hi[4 * g + 2] = h4.z, hi[4 * g + 3] = h4.w;
+          lo[4 * g] = l4.x, lo[4 * g + 1] = l4.y, lo[4 * g + 2] = l4.z, lo[4 * g + 3] = l4.w;
+        }
+        tmem_st32(tmem + lane_base + L::kColQhi + c * 32, hi);
+        tmem_st32(tmem + lane_base + L::kColQlo + c * 32, lo);
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
       mbar_arrive(&bars[L::kBarQReady]);
     }
     for (int j = 0; j < nt && ok; ++j) {
       const int sk = j % L::kKStages;
       if (!(ok = mbar_wait(&bars[L::kBarKFull + sk], (j / L::kKStages) & 1, wc))) break;
-      tf32_split_tile(smem + L::kOffKhi + sk * L::kKBytes, smem + L::kOffKlo + sk * L::kKBytes, L::kKBytes, st);
+      tf32_split_tile<L::kKBytes>(smem + L::kOffKhi + sk * L::kKBytes, smem + L::kOffKlo + sk * L::kKBytes, st);
       fence_proxy_async_smem();
       mbar_arrive(&bars[L::kBarKReady + sk]);
+    }
+  } else if (warp >= kTfWarpVSplit0) {
+    // ================================================================ V split warps
+    setmaxnreg_dec<kTfRegsOther>();
+    const int st = threadIdx.x - kTfWarpVSplit0 * 32;
+    // the first V^T tiles overwrite the Q staging area: its split must be done
+    bool ok = mbar_wait(&bars[L::kBarQReady], 0, wc);
+    for (int j = 0; j < nt && ok; ++j) {
       const int sv = j % L::kVRawStages, stv = j % L::kVtStages;
       if (!(ok = mbar_wait(&bars[L::kBarVFull + sv], (j / L::kVRawStages) & 1, wc))) break;
       if (j >= L::kVtStages && !(ok = mbar_wait(&bars[L::kBarVtEmpty + stv], ((j / L::kVtStages) - 1) & 1, wc)))
@@ -444,6 +501,7 @@ __global__ void __launch_bounds__(kTfThreads, 1) pba_attn_tf32_sm100_kernel(cons
     }
   } else {
     // ================================================================ softmax warps
+    setmaxnreg_inc<kTfRegsSoftmax>();
     const int t = threadIdx.x;  // query row inside the tile
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const uint32_t tS = tmem + lane_base + kTfColS;
@@ -543,26 +601,25 @@ __global__ void __launch_bounds__(kTfThreads, 1) pba_attn_tf32_sm100_kernel(cons
         for (int c = 0; c < w; ++c) ps[c] += ps[c + w];
       l += ps[0];
 
-      // P(j) overwrites the buffer that P V(j-2) read
-      if (j >= 2 && !(ok = warp_wait(&bars[L::kBarPFree + buf], ((j >> 1) - 1) & 1, wc))) break;
-      if (j >= 1 && __any_sync(0xffffffffu, need)) {
-        // rescale this warp's rows of O once P V(j-1) is done (lanes without
-        // a new maximum use 1)
-        const int jp = j - 1;
-        if (!(ok = warp_wait(&bars[L::kBarPFree + (jp & 1)], (jp >> 1) & 1, wc))) break;
+      // P(j) overwrites the P that P V(j-1) read, and a rescale of O needs
+      // P V(j-1) done as well
+      if (j >= 1) {
+        if (!(ok = warp_wait(&bars[L::kBarPDone], (j - 1) & 1, wc))) break;
         tc_fence_after_sync();
+        if (__any_sync(0xffffffffu, need)) {
+          // rescale this warp's rows of O (lanes without a new maximum use 1)
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + c, o);
-          tmem_wait_ld();
-          reg_fence(o);
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c, o);
+            tmem_wait_ld();
+            reg_fence(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + c, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + c, o);
+          }
         }
       }
-      tc_fence_after_sync();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t hi[32], lo[32];
@@ -572,19 +629,16 @@ __global__ void __launch_bounds__(kTfThreads, 1) pba_attn_tf32_sm100_kernel(cons
           hi[e] = to_tf32(v);
           lo[e] = to_tf32(v - __uint_as_float(hi[e]));
         }
-        tmem_st32(tPhi + buf * kTfBN + half * 32, hi);
-        tmem_st32(tPlo + buf * kTfBN + half * 32, lo);
+        tmem_st32(tPhi + half * 32, hi);
+        tmem_st32(tPlo + half * 32, lo);
       }
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&bars[L::kBarPFull + buf]);
+      mbar_arrive(&bars[L::kBarPFull]);
     }
 
     // ---------------------------------------------------------------- epilogue
-    if (ok) {
-      const int jl = nt - 1;  // the last P V: every earlier one is done too
-      ok = warp_wait(&bars[L::kBarPFree + (jl & 1)], (jl >> 1) & 1, wc);
-    }
+    if (ok) ok = warp_wait(&bars[L::kBarPDone], (nt - 1) & 1, wc);  // the last P V
     if (ok) {
       tc_fence_after_sync();
       float o[D];

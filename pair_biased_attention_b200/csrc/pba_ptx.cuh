@@ -363,12 +363,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // fp32 -> tf32, rounded to nearest (ties away from zero): the result is an
-// fp32 bit pattern whose 13 low mantissa bits are zero.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
+// fp32 bit pattern whose 13 low mantissa bits are zero.  Adding half of the
+// dropped field to the sign-magnitude bits and clearing the field rounds the
+// magnitude (a carry moves into the exponent, as rounding up should); two
+// integer operations on the full-rate pipes.  Finite inputs and infinities
+// only (a NaN whose payload lies in the low bits would become an infinity).
+__device__ __forceinline__ uint32_t to_tf32(float x) { return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u; }
 
 // tanh on the MUFU unit (tanh.approx.f32, an approximation with an error of
 // order 2^-11).
