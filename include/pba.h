@@ -51,7 +51,9 @@
  * multiple of 8 elements.  For pba_partial the caller points k, v, bias and
  * key_mask at the block's first key, so the block start must keep those rules
  * (a multiple of 8 keys).  The fp32 path has no alignment rule beyond natural
- * float alignment.
+ * float alignment: calls whose q, k, v, bias and out bases are 16-byte
+ * aligned and whose non-unit strides are multiples of 4 elements run on the
+ * tensor cores, the others on the CUDA cores (same results to about 1e-5).
  */
 #ifndef PBA_H
 #define PBA_H
@@ -87,10 +89,12 @@ typedef enum { PBA_TRI_STARTING = 0, PBA_TRI_ENDING = 1 } pba_tri_orient;
  *   Nq, Nk     query rows and keys (>= 0; Nk = 0 makes every row empty)
  *   D          head dimension: 32 or 64 (bf16 and fp32)
  *   dtype      pba_dtype of q, k, v, bias and of pba_forward's `out`.  bf16
- *              runs on the tensor cores; fp32 is the reference-precision
- *              path (CUDA cores, one warp per query row, fp32 end to end,
- *              about 1e-5 from the exact result): meant for checks and small
- *              problems, orders of magnitude slower than bf16 at size.
+ *              runs on the tensor cores (kind::f16).  fp32 keeps fp32-level
+ *              accuracy (about 1e-5 from the exact result): on the tensor
+ *              cores as kind::tf32 with each operand split into a tf32 high
+ *              and low part (three products per product, about six times
+ *              slower than bf16 at size), or, for rows the tile loads cannot
+ *              address, one warp per query row on the CUDA cores.
  *   softmax_scale  tau; 0 selects 1/sqrt(D).  The bias is added unscaled.
  *   *_stride   strides in ELEMENTS of the (b, h, n) axes; the d axis (and
  *              the key axis of the bias) has stride 1.

@@ -186,8 +186,9 @@ def pba_forward(q, k, v, bias, key_mask=None, out=None, lse=None, softmax_scale=
     """O (and the natural-log log-sum-exp) of pair-biased attention over all
     keys.  q [B,H,Nq,D], k/v [B,H,Nk,D], bias [B|1,H|1,Nq,Nk] (bf16 or fp32, all
     the same dtype), key_mask [B,Nk] uint8 (1 = key takes part) or None.
-    bf16 runs on the tensor cores; fp32 is the reference-precision path on the
-    CUDA cores (fp32 end to end), meant for checks and small problems."""
+    bf16 runs on the tensor cores; fp32 keeps fp32-level accuracy, on the
+    tensor cores as three tf32 products per product (high and low parts of
+    each operand) when the rows are 16-byte aligned, else on the CUDA cores."""
     for n, t in (("q", q), ("k", k), ("v", v), ("bias", bias)):
         _cuda(n, t, q.dtype)
     _cuda("key_mask", key_mask, torch.uint8)

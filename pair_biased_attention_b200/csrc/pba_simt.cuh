@@ -1,7 +1,8 @@
 // pba_simt.cuh -- the CUDA-core kernels of the library:
 //   * pba_attn_f32_kernel: pair-biased attention in fp32 for fp32 inputs
-//     (one warp per query row, exact expf, fp32 accumulation), the reference-
-//     precision path; the bf16 path runs on the tensor cores.
+//     whose rows the tile loads cannot address (one warp per query row,
+//     expf, fp32 accumulation); aligned fp32 inputs run on the tensor cores
+//     (pba_attn_tf32_sm100.cuh).
 //   * softmax_merge_kernel: the tiled-softmax merge of key-block partials
 //     ("Fold-CP: A Context Parallelism Framework for Biomolecular Modeling",
 //     Figure 2 (a) and (c)), a bandwidth-bound pass with 16-byte vector loads.
