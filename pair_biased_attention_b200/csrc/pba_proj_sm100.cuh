@@ -11,9 +11,8 @@
 //
 // Persistent, one CTA per SM, 192 threads:
 //   warps 0-3  epilogue: thread t owns pair row t of the tile (TMEM lane t);
-//              reads the fp32 accumulators, writes bf16 rows of q, k, v, g,
-//              and forms the H bias columns from the z tile in shared memory
-//              on the CUDA cores
+//              reads the fp32 accumulators, writes bf16 rows of q, k, v, g
+//              and the row's H bias values
 //   warp 4     TMA producer: W once (resident, 128 KB at c = 128), then one
 //              128-row z tile per stage of a 2-stage ring
 //   warp 5     allocates Tensor Memory and issues every tcgen05.mma
@@ -21,7 +20,11 @@
 // v|g of a tile, so that the epilogue of one half overlaps the MMAs of the
 // other.  Each half is c/16 MMAs of M128 N256 K16: A = the z tile (K-major,
 // 128-byte swizzle), B = four 64-column slabs of W (MN-major, 128-byte
-// swizzle, slabs LBO apart).
+// swizzle, slabs LBO apart).  The bias columns are c/16 more MMAs of
+// M128 N16 K16 against W_b^T (K-major, H rows padded to 16), issued after
+// the v|g half into the first 16 columns of the q|k half once the epilogue
+// has read them; the epilogue reads the bias after the rest of q|k and only
+// then frees that half for the next tile.
 #pragma once
 
 #include <cuda.h>
@@ -57,8 +60,11 @@ struct ProjLayout {
   static constexpr int kOffW = 0;
   static constexpr int kZStageMax = kProjRows * kProjMaxC * 2;  // one z tile at c = 128
   static constexpr int kOffZ = kOffW + kSlabs * kSlabMax;
-  static constexpr int kOffWb = kOffZ + kProjZStages * kZStageMax;  // W_b as fp32 [c][H]
-  static constexpr int kWbMax = kProjMaxC * 8 * 4;
+  // W_b^T as the bias MMA's B operand: [16 rows (h, zero past H)][c] bf16,
+  // K-major, 128-byte swizzle, one 2 KB block per 64 columns of c
+  static constexpr int kOffWb = kOffZ + kProjZStages * kZStageMax;
+  static constexpr int kWbChunkBytes = 16 * 128;
+  static constexpr int kWbMax = (kProjMaxC / 64) * kWbChunkBytes;
   // output staging: 32-column chunks of a tile ([128 rows][64 bytes], 64-byte
   // swizzle), three buffers so that one barrier per chunk suffices
   static constexpr int kStageBufs = 3;
@@ -70,7 +76,9 @@ struct ProjLayout {
   static constexpr int kBarZEmpty = kBarZFull + kProjZStages;
   static constexpr int kBarAccFull = kBarZEmpty + kProjZStages;
   static constexpr int kBarAccEmpty = kBarAccFull + 2;
-  static constexpr int kBarDrain = kBarAccEmpty + 2;
+  static constexpr int kBarBiasSlot = kBarAccEmpty + 2;  // the epilogue has read columns [0, 64) of q|k
+  static constexpr int kBarBiasFull = kBarBiasSlot + 1;  // the bias MMAs are done
+  static constexpr int kBarDrain = kBarBiasFull + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffAbort = kOffTmemSlot + 4;
@@ -87,7 +95,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kOffBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kOffTmemSlot);
   int *abort_flag = reinterpret_cast<int *>(smem + L::kOffAbort);
-  float *wb_s = reinterpret_cast<float *>(smem + L::kOffWb);
+  uint8_t *wb_s = smem + L::kOffWb;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -99,18 +107,27 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
     mbar_init(&bars[L::kBarW], 1);
     for (int s = 0; s < kProjZStages; ++s) {
       mbar_init(&bars[L::kBarZFull + s], 1);
-      mbar_init(&bars[L::kBarZEmpty + s], kProjRows + 1);  // every epilogue thread + the MMA commit
+      mbar_init(&bars[L::kBarZEmpty + s], 1);  // the MMA commit after the tile's last MMAs
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&bars[L::kBarAccFull + h], 1);
       mbar_init(&bars[L::kBarAccEmpty + h], kProjRows);
     }
+    mbar_init(&bars[L::kBarBiasSlot], kProjRows);
+    mbar_init(&bars[L::kBarBiasFull], 1);
     mbar_init(&bars[L::kBarDrain], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // W_b in fp32, read by the epilogue threads
-  for (int i = threadIdx.x; i < c * kH; i += kProjThreads) wb_s[i] = __uint_as_float(uint32_t(p.wb[i]) << 16);
+  // W_b^T into its swizzled K-major tile: element (h, k) in block k / 64, row
+  // h, 16-byte granule ((k % 64) / 8) ^ (h % 8); rows h >= H are zero
+  for (int i = threadIdx.x; i < 16 * c; i += kProjThreads) {
+    const int hh = i / c, k = i % c;
+    const uint16_t v = hh < kH ? p.wb[k * kH + hh] : uint16_t(0);
+    *reinterpret_cast<uint16_t *>(wb_s + (k >> 6) * L::kWbChunkBytes + hh * 128 + ((((k & 63) >> 3) ^ (hh & 7)) << 4) +
+                                  (k & 7) * 2) = v;
+  }
+  fence_proxy_async_smem();
   if (warp == 5) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -185,7 +202,23 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
           }
           tc_commit(&bars[L::kBarAccFull + hf]);
         }
-        if (ok) tc_commit(&bars[L::kBarZEmpty + s]);
+        // the bias columns, into the first 16 columns of q|k once the
+        // epilogue has read them: A = the z tile, B = W_b^T (K-major)
+        if (ok) ok = mbar_wait(&bars[L::kBarBiasSlot], it & 1, wc);
+        if (ok) {
+          tc_fence_after_sync();
+          const uint32_t zbase = sZ + s * L::kZStageMax;
+          const uint32_t sWb = smem_u32(smem + L::kOffWb);
+          const uint32_t idesc_b = idesc_bf16_f32(kProjRows, 16, false);
+#pragma unroll 4
+          for (int kk = 0; kk < c / 16; ++kk) {
+            const uint32_t alo = smem_desc_lo(zbase + (kk >> 2) * (kProjRows * 128) + (kk & 3) * 32, 16);
+            const uint32_t blo = smem_desc_lo(sWb + (kk >> 2) * L::kWbChunkBytes + (kk & 3) * 32, 16);
+            mma_bf16_ss(tmem, desc_join(alo, kHi), desc_join(blo, kHi), idesc_b, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars[L::kBarBiasFull]);
+          tc_commit(&bars[L::kBarZEmpty + s]);
+        }
       }
       tc_commit(&bars[L::kBarDrain]);
       mbar_wait(&bars[L::kBarDrain], 0, wc_drain);
@@ -198,41 +231,8 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
     int it = 0;
     int sc = 0;  // output chunks staged
     for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
-      const int s = it % kProjZStages;
       const int64_t r = int64_t(tile) * kProjRows + t;
       const bool live = r < p.rows;
-      // bias columns on the CUDA cores from the z row in shared memory
-      // The four warps leave a wait together (the staging below uses a named
-      // barrier, which has no time limit).
-      ok = named_bar_and(2, kProjRows, mbar_wait<false>(&bars[L::kBarZFull + s], (it / kProjZStages) & 1, wc));
-      if (!ok) break;
-      {
-        float acc[kH];
-#pragma unroll
-        for (int h = 0; h < kH; ++h) acc[h] = 0.f;
-        const uint8_t *zt = smem + L::kOffZ + s * L::kZStageMax;
-        for (int bx = 0; bx < c / 64; ++bx) {
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint4 zv = *reinterpret_cast<const uint4 *>(zt + bx * (kProjRows * 128) + t * 128 + ((ch ^ (t & 7)) << 4));
-            const uint32_t wv[4] = {zv.x, zv.y, zv.z, zv.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int cc = bx * 64 + ch * 8 + 2 * e;
-              const float z0 = bf16lo_to_f32(wv[e]), z1 = bf16hi_to_f32(wv[e]);
-#pragma unroll
-              for (int h = 0; h < kH; ++h) acc[h] = fmaf(z1, wb_s[(cc + 1) * kH + h], fmaf(z0, wb_s[cc * kH + h], acc[h]));
-            }
-          }
-        }
-        if (live)
-#pragma unroll
-          for (int h = 0; h < kH; ++h) {
-            const uint32_t bits = pack_bf16x2(acc[h], 0.f) & 0xFFFFu;
-            p.bias[int64_t(h) * p.rows + r] = uint16_t(bits);
-          }
-      }
-      mbar_arrive(&bars[L::kBarZEmpty + s]);
       // q|k from half 0, v|g from half 1, as 32-column chunks: Tensor Memory ->
       // registers -> bf16 -> swizzled staging buffer -> one tensor store per
       // chunk (issued by thread 0 after a barrier of the four warps).
@@ -248,9 +248,13 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
           tmem_wait_ld();
           reg_fence(a[0]);
           reg_fence(a[1]);
-          if (cc == 6) {
+          if (hf == 0 && cc == 0) {
             tc_fence_before_sync();
-            mbar_arrive(&bars[L::kBarAccEmpty + hf]);  // this half of Tensor Memory is free
+            mbar_arrive(&bars[L::kBarBiasSlot]);  // columns [0, 64) read: the bias MMAs may write there
+          }
+          if (hf == 1 && cc == 6) {
+            tc_fence_before_sync();
+            mbar_arrive(&bars[L::kBarAccEmpty + 1]);  // this half of Tensor Memory is free
           }
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
@@ -277,6 +281,22 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
             }
             ++sc;
           }
+        }
+        if (hf == 0) {
+          // the row's bias values, then q|k's columns are free for the next tile
+          ok = named_bar_and(2, kProjRows, mbar_wait<false>(&bars[L::kBarBiasFull], it & 1, wc));
+          if (!ok) break;
+          tc_fence_after_sync();
+          uint32_t bv[16];
+          tmem_ld16(tmem + lane_base, bv);
+          tmem_wait_ld();
+          reg_fence(bv);
+          tc_fence_before_sync();
+          mbar_arrive(&bars[L::kBarAccEmpty + 0]);
+          if (live)
+#pragma unroll
+            for (int h = 0; h < kH; ++h)
+              p.bias[int64_t(h) * p.rows + r] = uint16_t(pack_bf16x2(__uint_as_float(bv[h]), 0.f) & 0xFFFFu);
         }
       }
     }
