@@ -83,10 +83,12 @@ struct BwdLayout {
   static constexpr int kOffStep0 = kOffFix1 + kTileBytes;                   // [stage]
   static constexpr int kOffStep1 = kOffStep0 + kStages * kTileBytes;        // [stage]
   static constexpr int kOffBias = kOffStep1 + kStages * kTileBytes;         // [stage]
-  // kernel B: log2-scaled lse and Delta of the step's 128 query columns,
-  // double-buffered by step parity
+  // per-step column data, one copy per compute warp (so that a warp needs no
+  // barrier with the others of its warpgroup), double-buffered by step
+  // parity: A: 32 keep words; B: -lse log2(e) and -Delta of 64 query columns
+  static constexpr int kRowvWarpFloats = kBwdTile;
   static constexpr int kOffRowv = kOffBias + kStages * kBiasBytes;
-  static constexpr int kOffBar = kOffRowv + 2 * 2 * kBwdTile * 4;
+  static constexpr int kOffBar = kOffRowv + 2 * (4 * kBwdComputeGroups) * kRowvWarpFloats * 4;
   static constexpr int kBarFixFull = 0;
   static constexpr int kBarStepFull = 1;                       // [stage]
   static constexpr int kBarStepEmpty = kBarStepFull + kStages;  // [stage]
@@ -289,25 +291,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       key_ok = r < p.Nk && (mrow == nullptr || mrow[r] != 0);
     }
     // Column data of a step, loaded from global memory one step ahead so
-    // that the loads' latency overlaps a step of work.  A: the mask bytes of
-    // this thread's key pair (threads t < 32); B: lse and Delta of this
-    // thread's query column (threads t < 64).
+    // that the loads' latency overlaps a step of work; every warp loads the
+    // data of its warpgroup's columns for itself.  A: the mask bytes of key
+    // pair `lane`; B: lse and Delta of query columns `lane` and `lane + 32`.
     uint32_t nm0 = 1u, nm1 = 1u;
-    float nlse = 0.f, ndelta = 0.f;
+    float nlse[2] = {0.f, 0.f}, ndelta[2] = {0.f, 0.f};
     auto load_cols = [&](int step) {
       const int o = step * kBwdTile;
       if (!kB) {
-        if (t < kBwdTile / 4 && mrow != nullptr) {
-          const int key = o + 2 * (g * (kBwdTile / 4) + t);
+        if (mrow != nullptr) {
+          const int key = o + 2 * (g * (kBwdTile / 4) + lane);
           nm0 = key < p.Nk ? uint32_t(mrow[key]) : 0u;
           nm1 = key + 1 < p.Nk ? uint32_t(mrow[key + 1]) : 0u;
         }
-      } else if (t < kBwdTile / 2) {
-        const int qi = o + g * (kBwdTile / 2) + t;
-        if (qi < p.Nq) {
-          const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
-          nlse = p.lse[at];
-          ndelta = p.delta[at];
+      } else {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int qi = o + g * (kBwdTile / 2) + lane + 32 * e;
+          if (qi < p.Nq) {
+            const int64_t at = int64_t(b) * p.row_sb + int64_t(h) * p.row_sh + qi;
+            nlse[e] = p.lse[at];
+            ndelta[e] = p.delta[at];
+          }
         }
       }
     };
@@ -317,35 +322,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       const int s = it % L::kStages;
       const int o0 = it * kBwdTile;
       const uint32_t cm0 = nm0, cm1 = nm1;
-      const float clse = nlse, cdelta = ndelta;
+      const float clse[2] = {nlse[0], nlse[1]}, cdelta[2] = {ndelta[0], ndelta[1]};
       if (it + 1 < nsteps) load_cols(it + 1);
-      // S, dP and the step's tiles.  The waits only set ok; the warpgroup
-      // leaves together at the barrier below.
+      // S, dP and the step's tiles.  The waits only set ok; the warp leaves
+      // together at the vote below.
       ok = mbar_wait<false>(&bars[L::kBarSFull], it & 1, wc);
       if (ok) ok = mbar_wait<false>(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
       const uint8_t *bt = smem + L::kOffBias + s * L::kBiasBytes;
-      // Per-step column data in shared memory (double-buffered by step
-      // parity); each warpgroup writes and reads only its own 64 columns, and
-      // its barrier also makes its warps leave the loop together.  A: one
-      // keep word per key pair (0xFFFF per kept half: masked keys and keys
-      // past Nk turn into bf16 -inf in the bias).  B: -lse*log2(e) and -Delta
-      // of the query columns (columns past Nq get -lse = -inf, so P = 0 there).
-      float *rv = reinterpret_cast<float *>(smem + L::kOffRowv) + (it & 1) * 2 * kBwdTile;
+      // Per-step column data in this warp's own shared-memory copy
+      // (double-buffered by step parity), written and read by the warp alone.
+      // A: one keep word per key pair of the warpgroup's 64 columns (0xFFFF
+      // per kept half: masked keys and keys past Nk turn into bf16 -inf in
+      // the bias).  B: -lse*log2(e) at [0, 64) and -Delta at [64, 128) for
+      // the warpgroup's query columns (columns past Nq get -lse = -inf, so
+      // P = 0 there).
+      float *rv = reinterpret_cast<float *>(smem + L::kOffRowv) +
+                  ((it & 1) * (4 * kBwdComputeGroups) + warp) * L::kRowvWarpFloats;
       if (!kB) {
-        if (t < kBwdTile / 4) {
-          const int pr = g * (kBwdTile / 4) + t;  // key pair of the step
-          const int key = o0 + 2 * pr;
-          const uint32_t keep = ((key < p.Nk && cm0 != 0u) ? 0x0000FFFFu : 0u) |
-                                ((key + 1 < p.Nk && cm1 != 0u) ? 0xFFFF0000u : 0u);
-          reinterpret_cast<uint32_t *>(rv)[pr] = keep;
+        const int key = o0 + 2 * (g * (kBwdTile / 4) + lane);  // key pair `lane` of the warpgroup
+        const uint32_t keep = ((key < p.Nk && cm0 != 0u) ? 0x0000FFFFu : 0u) |
+                              ((key + 1 < p.Nk && cm1 != 0u) ? 0xFFFF0000u : 0u);
+        reinterpret_cast<uint32_t *>(rv)[lane] = keep;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = lane + 32 * e;  // query column of the warpgroup's half
+          const int qi = o0 + g * (kBwdTile / 2) + col;
+          rv[col] = qi >= p.Nq ? -INFINITY : (clse[e] == -INFINITY ? 0.f : -clse[e] * l2e);  // see the A side
+          rv[kBwdTile / 2 + col] = qi < p.Nq ? -cdelta[e] : 0.f;
         }
-      } else if (t < kBwdTile / 2) {
-        const int col = g * (kBwdTile / 2) + t;  // query column of the step
-        const int qi = o0 + col;
-        rv[col] = qi >= p.Nq ? -INFINITY : (clse == -INFINITY ? 0.f : -clse * l2e);  // see the A side
-        rv[kBwdTile + col] = qi < p.Nq ? -cdelta : 0.f;
       }
-      ok = named_bar_and(1 + g, kBwdTile, ok);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after_sync();
       const float2 cs2 = make_float2(c_s, c_s), l2e2 = make_float2(l2e, l2e);
@@ -383,7 +391,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
               const int box = c >> 6, chunk = (c & 63) >> 3;
               const uint4 w4 = *reinterpret_cast<const uint4 *>(bt + box * (L::kBiasBytes / 2) + t * 128 +
                                                                 ((chunk ^ (t & 7)) << 4));
-              const uint4 k4 = reinterpret_cast<const uint4 *>(rv)[c8 + hf * 8];
+              const uint4 k4 = reinterpret_cast<const uint4 *>(rv)[c8];
               const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -394,10 +402,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
               }
             } else {
               // plain [query][key] tile: queries c .. c+7 of key column t
-              const float4 la = *reinterpret_cast<const float4 *>(rv + c);
-              const float4 lb = *reinterpret_cast<const float4 *>(rv + c + 4);
-              const float4 da = *reinterpret_cast<const float4 *>(rv + kBwdTile + c);
-              const float4 db = *reinterpret_cast<const float4 *>(rv + kBwdTile + c + 4);
+              const int cl = c8 * 8;  // the columns' place in the warp's copy
+              const float4 la = *reinterpret_cast<const float4 *>(rv + cl);
+              const float4 lb = *reinterpret_cast<const float4 *>(rv + cl + 4);
+              const float4 da = *reinterpret_cast<const float4 *>(rv + kBwdTile / 2 + cl);
+              const float4 db = *reinterpret_cast<const float4 *>(rv + kBwdTile / 2 + cl + 4);
               const float2 lv[4] = {make_float2(la.x, la.y), make_float2(la.z, la.w), make_float2(lb.x, lb.y),
                                     make_float2(lb.z, lb.w)};
               const float2 dv[4] = {make_float2(da.x, da.y), make_float2(da.z, da.w), make_float2(db.x, db.y),
@@ -445,8 +454,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
             // the previous step's accumulating MMAs read G0/G1, which the
             // stores below overwrite: wait for them only now, so that they
             // overlap this quarter's arithmetic
-            ok = mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc);
-            ok = named_bar_and(1 + g, kBwdTile, ok);
+            ok = __all_sync(0xffffffffu, mbar_wait<false>(&bars[L::kBarGDone], (it - 1) & 1, wc));
             if (!ok) break;
             tc_fence_after_sync();
           }
@@ -466,8 +474,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     }
     // -------------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait<false>(&bars[L::kBarGDone], (nsteps - 1) & 1, wc);
-    // the warpgroup's threads all get here; the loads below are warp-collective
-    ok = named_bar_and(1 + g, kBwdTile, ok);
+    // the loads below are warp-collective: the warp leaves the wait as one
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after_sync();
       const int nrows = kB ? p.Nk : p.Nq;
