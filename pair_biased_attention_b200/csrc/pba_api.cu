@@ -710,7 +710,8 @@ pba_status tri_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, const vo
     void *const dst[4] = {q, k, v, g};
     const uint64_t dims[4] = {uint64_t(pba::kProjCols / 4), uint64_t(rows), 1, 1};
     const int64_t st[3] = {int64_t(pba::kProjCols / 4) * 2, 0, 0};
-    const uint32_t box[4] = {32, uint32_t(pba::kProjRows), 1, 1};
+    // one warp's 32 rows of a 32-column chunk per tensor store
+    const uint32_t box[4] = {32, 32, 1, 1};
     if (!make_map(&p.tm_out[m], dst[m], dims, st, box, CU_TENSOR_MAP_SWIZZLE_64B)) return PBA_ERR_INVALID_ARG;
   }
   p.rows = rows;

@@ -43,7 +43,7 @@ constexpr int kProjMaxC = 128;
 struct ProjParams {
   CUtensorMap tm_z;  // z [rows][c] bf16, box {64, 128}
   CUtensorMap tm_w;  // W [c][512] bf16, box {64, c}
-  CUtensorMap tm_out[4];  // q, k, v, g [rows][128] bf16, box {32, 128}, 64-byte swizzle (stores)
+  CUtensorMap tm_out[4];  // q, k, v, g [rows][128] bf16, box {32, 32}, 64-byte swizzle (stores)
   int64_t rows;      // N*N
   int32_t c;         // 64 or 128
   int32_t n_tiles;   // ceil(rows / 128)
@@ -66,7 +66,8 @@ struct ProjLayout {
   static constexpr int kWbChunkBytes = 16 * 128;
   static constexpr int kWbMax = (kProjMaxC / 64) * kWbChunkBytes;
   // output staging: 32-column chunks of a tile ([128 rows][64 bytes], 64-byte
-  // swizzle), three buffers so that one barrier per chunk suffices
+  // swizzle; warp w's rows are the 2 KB at 2 KB w, stored by the warp on its
+  // own), three buffers
   static constexpr int kStageBufs = 3;
   static constexpr int kStageBytes = kProjRows * 64;
   static constexpr int kOffStage = kOffWb + kWbMax;
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
       // registers -> bf16 -> swizzled staging buffer -> one tensor store per
       // chunk (issued by thread 0 after a barrier of the four warps).
       for (int hf = 0; hf < 2 && ok; ++hf) {
-        ok = named_bar_and(2, kProjRows, mbar_wait<false>(&bars[L::kBarAccFull + hf], it & 1, wc));
+        ok = __all_sync(0xffffffffu, mbar_wait<false>(&bars[L::kBarAccFull + hf], it & 1, wc));
         if (!ok) break;
         tc_fence_after_sync();
 #pragma unroll 1
@@ -269,22 +270,23 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
               *reinterpret_cast<uint4 *>(buf + t * 64 + ((j ^ ((t >> 1) & 3)) << 4)) = v;
             }
             fence_proxy_async_smem();
-            named_bar_sync(1, kProjRows);
-            if (t == 0) {
+            __syncwarp();
+            if (lane == 0) {
               const int m = chunk >> 2;  // 0 q, 1 k, 2 v, 3 g
               const CUtensorMap *map = m == 0 ? &p.tm_out[0] : m == 1 ? &p.tm_out[1] : m == 2 ? &p.tm_out[2] : &p.tm_out[3];
-              tma_store_4d(map, buf, (chunk & 3) * 32, tile * kProjRows, 0, 0);
+              tma_store_4d(map, buf + warp * 2048, (chunk & 3) * 32, tile * kProjRows + warp * 32, 0, 0);
               bulk_commit_group();
               // the buffer the next chunk but one writes is free once this
               // chunk's predecessor has been read out
               bulk_wait_group_read<1>();
             }
+            __syncwarp();
             ++sc;
           }
         }
         if (hf == 0) {
           // the row's bias values, then q|k's columns are free for the next tile
-          ok = named_bar_and(2, kProjRows, mbar_wait<false>(&bars[L::kBarBiasFull], it & 1, wc));
+          ok = __all_sync(0xffffffffu, mbar_wait<false>(&bars[L::kBarBiasFull], it & 1, wc));
           if (!ok) break;
           tc_fence_after_sync();
           uint32_t bv[16];
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(kProjThreads, 1) pba_proj_sm100_kernel(const _
         }
       }
     }
-    if (t == 0) bulk_wait_group_all();  // staging buffers are read and the rows written
+    if (lane == 0) bulk_wait_group_all();  // this warp's staging buffers are read and its rows written
   }
 
   tc_fence_before_sync();
