@@ -767,7 +767,8 @@ pba_status tri_out_proj_forward(int64_t N, int64_t c, int64_t H, int64_t D, cons
   {
     const uint64_t dims[4] = {uint64_t(c), uint64_t(rows), 1, 1};
     const int64_t st[3] = {c * 2, 0, 0};
-    const uint32_t box[4] = {32, uint32_t(pba::kOprojRows), 1, 1};
+    // one warp's 32 rows of a 32-column chunk per tensor store
+    const uint32_t box[4] = {32, 32, 1, 1};
     if (!make_map(&p.tm_out, out, dims, st, box, CU_TENSOR_MAP_SWIZZLE_64B)) return PBA_ERR_INVALID_ARG;
   }
   p.rows = rows;

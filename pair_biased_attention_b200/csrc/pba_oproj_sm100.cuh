@@ -35,7 +35,7 @@ constexpr int kOprojStages = 4;
 struct OprojParams {
   CUtensorMap tm_o;    // o [rows][128] bf16, box {64, 128}, 128-byte swizzle
   CUtensorMap tm_w;    // W_o [128][c] bf16, box {64, 128}, 128-byte swizzle
-  CUtensorMap tm_out;  // out [rows][c] bf16, box {32, 128}, 64-byte swizzle (stores)
+  CUtensorMap tm_out;  // out [rows][c] bf16, box {32, 32}, 64-byte swizzle (stores, one warp's rows each)
   int64_t rows;        // N*N
   int32_t n_tiles;     // ceil(rows / 128)
   int *err;
@@ -182,9 +182,8 @@ __global__ void __launch_bounds__(kOprojThreads, 1) pba_oproj_sm100_kernel(const
     int sc = 0;  // output chunks staged
     for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
       const int b = it & 1;
-      // The four warps leave a wait together (the staging below uses a named
-      // barrier, which has no time limit).
-      ok = named_bar_and(2, kOprojRows, mbar_wait<false>(&bars[L::kBarAccFull + b], (it >> 1) & 1, wc));
+      // the warp leaves the wait as one (the loads below are warp-collective)
+      ok = __all_sync(0xffffffffu, mbar_wait<false>(&bars[L::kBarAccFull + b], (it >> 1) & 1, wc));
       if (!ok) break;
       tc_fence_after_sync();
 #pragma unroll 1
@@ -208,18 +207,20 @@ __global__ void __launch_bounds__(kOprojThreads, 1) pba_oproj_sm100_kernel(const
           *reinterpret_cast<uint4 *>(buf + t * 64 + ((j ^ ((t >> 1) & 3)) << 4)) = v;
         }
         fence_proxy_async_smem();
-        named_bar_sync(1, kOprojRows);
-        if (t == 0) {
-          tma_store_4d(&p.tm_out, buf, ch * 32, tile * kOprojRows, 0, 0);
+        __syncwarp();
+        if (lane == 0) {
+          // this warp's 32 rows (the 2 KB at 2 KB warp of the buffer)
+          tma_store_4d(&p.tm_out, buf + warp * 2048, ch * 32, tile * kOprojRows + warp * 32, 0, 0);
           bulk_commit_group();
           // the buffer the chunk after next writes is free once this chunk's
           // predecessor has been read out
           bulk_wait_group_read<1>();
         }
+        __syncwarp();
         ++sc;
       }
     }
-    if (t == 0) bulk_wait_group_all();  // staging buffers are read and the rows written
+    if (lane == 0) bulk_wait_group_all();  // this warp's staging buffers are read and its rows written
   }
 
   tc_fence_before_sync();
