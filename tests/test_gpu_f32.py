@@ -135,3 +135,23 @@ def test_f32_apb2k_shape_sampled_rows(cuda_device):
         sel = lambda x: x[:, h:h + 1].index_select(2, rows_t)
         ref = oracle.pba(sel(q), k[:, h:h + 1], v[:, h:h + 1], sel(bias), mask)
         _check(f"f32 apb2k h={h}", sel(out), sel(lse), ref)
+
+
+def test_f32_strided_views_and_batch_broadcast_bias(cuda_device):
+    """Every other head of larger q, k, v tensors (head strides doubled), a
+    bias shared by the batch only (batch stride 0) and a partial over a key
+    block given as column views, all on the tensor-core path."""
+    qb, kb, vb, bias, mask = W.random_attn(2, 6, 140, 264, 64, dtype=torch.float32, seed=33, device=cuda_device,
+                                           mask_frac=0.1)
+    q, k, v = qb[:, ::2], kb[:, ::2], vb[:, ::2]
+    assert q.stride(1) == 2 * 140 * 64
+    b1 = bias[:1, ::2]  # [1, 3, 140, 264] -> batch stride 0 once expanded
+    _run("f32 strided", q, k, v, b1, mask)
+    # a key block of the same problem as column views (block start a multiple of 8 keys)
+    sl = slice(64, 200)
+    o_p, m_p, l_p = pba.pba_partial(q, k[:, :, sl], v[:, :, sl], b1[..., sl], mask[:, sl])
+    ref = oracle.pba_partial(q, k, v, b1.expand(2, 3, -1, -1), mask, k0=64, L=136)
+    assert np.abs(_np(o_p) - ref["o"]).max() <= F32_TOL
+    fin = ref["l"] > 0
+    lse_p = _np(m_p) + np.log(np.where(_np(l_p) > 0, _np(l_p), 1.0))
+    assert np.abs(lse_p[fin] - (ref["m"] + np.log(np.where(fin, ref["l"], 1.0)))[fin]).max(initial=0) <= F32_TOL
