@@ -923,6 +923,11 @@ pba_status pba_backward(const pba_attn_desc *d, const void *q, const void *k, co
     pba::BwdParams a = p;
     const uint32_t bbox[4] = {64, uint32_t(pba::kBwdTile), 1, 1};
     if (!make_map(&a.tm_bias, bias, bdims, bst, bbox, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
+    // dbias [B][H][Nq][Nk] (contiguous) as (Nk, Nq, H, B), one warp's 32 rows of 64 keys per store
+    const uint64_t ddims[4] = {uint64_t(Nk), uint64_t(Nq), uint64_t(H), uint64_t(B)};
+    const int64_t dst_[3] = {Nk * 2, Nq * Nk * 2, H * Nq * Nk * 2};
+    const uint32_t dbox[4] = {64, 32, 1, 1};
+    if (!make_map(&a.tm_dbias, dbias, ddims, dst_, dbox, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
     a.n_tiles = int((Nq + pba::kBwdTile - 1) / pba::kBwdTile);
     const int grid = int(B * H * a.n_tiles);
     e = (D == 64) ? launch_bwd<64, false>(a, grid, st) : launch_bwd<32, false>(a, grid, st);

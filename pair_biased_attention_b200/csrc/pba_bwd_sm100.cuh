@@ -52,6 +52,9 @@ struct BwdParams {
   // bf16, kernel A box {64, 128} 128-byte swizzle, kernel B box {128, 128}
   // no swizzle.
   CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_bias;
+  // A: dbias (Nk, Nq, H, B) bf16, box {64, 32} 128-byte swizzle: one warp's
+  // 32 rows of a 64-key half of a step, stored from the step's bias slot
+  CUtensorMap tm_dbias;
   int32_t B, H, Nq, Nk;
   int32_t n_tiles;      // A: ceil(Nq/128), B: ceil(Nk/128) per (b, h)
   int32_t bias_h_bcast, bias_b_bcast;  // bias head / batch stride 0 (map extent 1)
@@ -134,8 +137,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     mbar_init(&bars[L::kBarFixFull], 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[L::kBarStepFull + s], 1);
-      // the MMA commit + each compute warpgroup (bias, row values)
-      mbar_init(&bars[L::kBarStepEmpty + s], 1 + kBwdComputeGroups);
+      // the MMA commit + each compute warp (A: its dbias store has read the
+      // slot) or warpgroup (B: its bias half is read)
+      mbar_init(&bars[L::kBarStepEmpty + s], 1 + (kB ? kBwdComputeGroups : 4 * kBwdComputeGroups));
     }
     mbar_init(&bars[L::kBarSFull], 1);
     mbar_init(&bars[L::kBarSFree], kBwdComputeGroups * kBwdTile);
@@ -434,20 +438,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
             }
           }
           if (!kB) {
-            // dbias row segment (32 keys) and dS into Tensor Memory
-            const int key0 = o0 + hf * 64 + qt * 32;
-            if (r < p.Nq) {
-              uint16_t *dst = p.dbias + int64_t(b) * p.db_sb + int64_t(h) * p.db_sh + int64_t(r) * p.db_sn + key0;
-              if (key0 + 32 <= p.Nk) {
+            // dbias: this row's dS over the quarter's 32 keys, written in
+            // place of the bias values it came from (same swizzled 16-byte
+            // chunks of the step's bias slot, read by this thread alone); the
+            // warp stores its rows with one tensor store at the end of the step
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                  reinterpret_cast<uint4 *>(dst)[q] =
-                      make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
-              } else {
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                  if (key0 + e < p.Nk) dst[e] = uint16_t((e & 1) ? (dk[e >> 1] >> 16) : (dk[e >> 1] & 0xFFFFu));
-              }
+            for (int q = 0; q < 4; ++q) {
+              const int c = hf * 64 + qt * 32 + q * 8;
+              const int box = c >> 6, chunk = (c & 63) >> 3;
+              *reinterpret_cast<uint4 *>(const_cast<uint8_t *>(bt) + box * (L::kBiasBytes / 2) + t * 128 +
+                                         ((chunk ^ (t & 7)) << 4)) =
+                  make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
             }
           }
           if (qt == 0 && it > 0) {
@@ -470,7 +471,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&bars[L::kBarGFull]);
-      if (t == 0) mbar_arrive(&bars[L::kBarStepEmpty + s]);  // this warpgroup's bias half read
+      if (!kB) {
+        // the warp's 32 rows of dbias for its warpgroup's 64 keys: one tensor
+        // store from the slot (rows past Nq and keys past Nk are clipped);
+        // the slot is released once the store has read it
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int w4 = warp & 3;
+          tma_store_4d(&p.tm_dbias, bt + g * (L::kBiasBytes / 2) + w4 * 32 * 128, o0 + g * 64, row0 + 32 * w4, h,
+                       b);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();
+          mbar_arrive(&bars[L::kBarStepEmpty + s]);
+        }
+      } else if (t == 0) {
+        mbar_arrive(&bars[L::kBarStepEmpty + s]);  // this warpgroup's bias half read
+      }
     }
     // -------------------------------------------------------------- epilogue
     if (ok) ok = mbar_wait<false>(&bars[L::kBarGDone], (nsteps - 1) & 1, wc);
@@ -506,6 +523,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     }
   }
 
+  // the warps' dbias tensor stores are complete before the CTA ends
+  if (!kB && warp < kBwdWarpProducer && lane == 0) bulk_wait_group_all();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
