@@ -209,6 +209,13 @@ pba_status run_tc(const TcProblem &t, cudaStream_t stream) {
       if (!make_map(&p.tm_bias, t.bias, dims, st, box, CU_TENSOR_MAP_SWIZZLE_128B)) return PBA_ERR_INVALID_ARG;
     }
   }
+  if (t.D == 32 && t.epi == pba::kEpiForward) {
+    // the bf16 output rows, stored by warps of 32 rows from the staging buffer
+    const uint64_t dims[4] = {uint64_t(t.D), uint64_t(t.Nq), uint64_t(t.H), uint64_t(t.B)};
+    const int64_t st[3] = {t.out_s[2] * 2, t.out_s[1] * 2, t.out_s[0] * 2};
+    const uint32_t box[4] = {32, 32, 1, 1};
+    if (!make_map(&p.tm_out, t.out, dims, st, box, CU_TENSOR_MAP_SWIZZLE_64B)) return PBA_ERR_INVALID_ARG;
+  }
   p.B = t.B;
   p.H = t.H;
   p.Nq = t.Nq;

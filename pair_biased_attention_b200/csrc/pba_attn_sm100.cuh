@@ -57,6 +57,9 @@ enum Epilogue : int { kEpiForward = 0, kEpiPartial = 1 };
 
 struct AttnParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_bias;
+  // D = 32, forward: the bf16 output (D, Nq, H, B), box {32, 32} with the
+  // 64-byte swizzle, one warp's 32 rows per tensor store
+  CUtensorMap tm_out;
   int32_t B, H, Nq, Nk;
   int32_t n_qblocks;     // ceil(Nq / 256)
   int32_t n_units;       // B * H * n_qblocks
@@ -94,7 +97,12 @@ struct AttnLayout {
   static constexpr int kOffBias = kOffV + kKVStages * kKVBytes;
   // key-mask words: one u32 per key pair of a bias slot (0xFFFF per valid half)
   static constexpr int kOffMaskWords = kOffBias + kQTiles * kBiasStages * kBiasBytes;
-  static constexpr int kOffBar = kOffMaskWords + kQTiles * kBiasStages * (kBN / 2) * 4;
+  // D = 32: the forward epilogue's output rows, staged for tensor stores
+  // ([128 rows][64 bytes] per query tile, 64-byte swizzle); at D = 64 there is
+  // no room and the rows go straight to global memory
+  static constexpr bool kOutStaged = (D == 32);
+  static constexpr int kOffOut = kOffMaskWords + kQTiles * kBiasStages * (kBN / 2) * 4;
+  static constexpr int kOffBar = kOffOut + (kOutStaged ? kQTiles * kBM * kRowBytes : 0);
   // barriers
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQEmpty = 1;
@@ -647,6 +655,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       const Unit un = decode_unit(p, u);  // derived here so it is not live across the tile loop
       const int row = un.q0 + w * kBM + t;
       const int b = un.b, h = un.h;
+      if (kEpi == kEpiForward && L::kOutStaged) {
+        // the warp's staging rows were last read by the previous unit's store
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+      }
       if (row < p.Nq) {
         const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
         if (kEpi == kEpiForward) {
@@ -667,6 +680,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           }
           uint4 *op = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + b * p.out_sb + h * p.out_sh +
                                                 (int64_t)row * p.out_sn);
+          // staged rows: this thread's row of the warpgroup's buffer, 16-byte
+          // chunks swizzled by bits 7-8 of the row address
+          uint8_t *srow = smem + L::kOffOut + (w * kBM + t) * L::kRowBytes;
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) {
             uint32_t wv[4];
@@ -679,7 +695,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
               }
               wv[e] = pack_bf16x2(v0, v1);
             }
-            op[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            if (L::kOutStaged)
+              *reinterpret_cast<uint4 *>(srow + ((c ^ ((t >> 1) & 3)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            else
+              op[c] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
           }
           if (p.lse != nullptr)
             p.lse[b * p.lse_sb + h * p.lse_sh + (int64_t)row * p.lse_sn] = (l > 0.f) ? m_cur + logf(l) : -INFINITY;
@@ -694,7 +713,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           p.l_part[mi] = (l > 0.f) ? l * ex2_approx((m_cur - m_true) * kLog2e) : 0.f;
         }
       }
+      if (kEpi == kEpiForward && L::kOutStaged) {
+        // the warp's 32 rows with one tensor store (rows past Nq are clipped)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int wq = warp & 3;
+          tma_store_4d(&p.tm_out, smem + L::kOffOut + (w * kBM + 32 * wq) * L::kRowBytes, 0, un.q0 + w * kBM + 32 * wq,
+                       h, b);
+          bulk_commit_group();
+        }
+      }
     }
+    // the output stores are complete before the CTA ends
+    if (kEpi == kEpiForward && L::kOutStaged && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before_sync();
