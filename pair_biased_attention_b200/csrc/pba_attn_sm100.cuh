@@ -495,6 +495,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       float m_cur = -INFINITY;   // maximum used for P and l
       float m_true = -INFINITY;  // true running maximum
       float l = 0.f;
+      if (kGate && L::kOutStaged) {
+        // The gate row goes into this thread's output staging row while the
+        // unit's key tiles are processed; the epilogue reads it there and
+        // then overwrites it with the output.  The previous unit's tensor
+        // store must have read the rows first.
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        const Unit gu = decode_unit(p, u);
+        const int grow = gu.q0 + w * kBM + t;
+        uint8_t *srow = smem + L::kOffOut + (w * kBM + t) * L::kRowBytes;
+        if (grow < p.Nq) {
+          const uint8_t *src = reinterpret_cast<const uint8_t *>(p.gate + gu.b * p.gate_sb + gu.h * p.gate_sh +
+                                                                 (int64_t)grow * p.gate_sn);
+#pragma unroll
+          for (int c = 0; c < L::kRowBytes / 16; ++c) cp_async16(srow + ((c ^ ((t >> 1) & 3)) << 4), src + c * 16);
+        }
+        cp_async_commit();
+      }
       for (int j = 0; j < nt && ok; ++j, ++gt) {
         // The bias tile lands long before it is used: wait for it first and
         // start loading its first half from shared memory, so that those loads
@@ -655,8 +673,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       const Unit un = decode_unit(p, u);  // derived here so it is not live across the tile loop
       const int row = un.q0 + w * kBM + t;
       const int b = un.b, h = un.h;
-      if (kEpi == kEpiForward && L::kOutStaged) {
+      if (kEpi == kEpiForward && L::kOutStaged && !kGate) {
         // the warp's staging rows were last read by the previous unit's store
+        // (with a gate this was waited for at the unit's start)
         if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
       }
@@ -667,9 +686,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           if (kGate) {
             const uint4 *gptr = reinterpret_cast<const uint4 *>(p.gate + b * p.gate_sb + h * p.gate_sh +
                                                                 (int64_t)row * p.gate_sn);
+            uint8_t *grow_s = smem + L::kOffOut + (w * kBM + t) * L::kRowBytes;
+            if (L::kOutStaged) cp_async_wait_all();
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {
-              const uint4 gv = gptr[c];
+              const uint4 gv = L::kOutStaged ? *reinterpret_cast<const uint4 *>(grow_s + ((c ^ ((t >> 1) & 3)) << 4))
+                                             : gptr[c];
               const uint32_t wv[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -725,8 +747,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         }
       }
     }
-    // the output stores are complete before the CTA ends
+    // the output stores and gate copies are complete before the CTA ends
     if (kEpi == kEpiForward && L::kOutStaged && lane == 0) bulk_wait_group_all();
+    if (kGate && L::kOutStaged) cp_async_wait_all();
   }
 
   tc_fence_before_sync();
