@@ -134,11 +134,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 // maximum is used consistently for P and l, so the result is unchanged and the
 // probabilities stay below 2^8.
 constexpr float kRescaleThreshold = 8.0f / kLog2e;
-// One key pair in kExpEmuEvery takes the software exp2 (0: none).  At D = 32
-// the exp2 unit is the tighter limit and a third of the pairs move to the FMA
-// pipe; at D = 64 the softmax is issue-bound and all pairs use the unit.
+// One key pair in kExpEmuEvery takes the software exp2 on the FMA pipe (0:
+// none).  Neither head dimension gains from it: at D = 64 the softmax is
+// issue-bound, and at D = 32 (triangle attention, tri1024) every share
+// measured was slower than none: one pair in four +2 to +4 %, one in three
+// +4 to +7 %, one in two +13 to +30 %.
 #ifndef PBA_EXP_EMU_EVERY_D32
-#define PBA_EXP_EMU_EVERY_D32 3
+#define PBA_EXP_EMU_EVERY_D32 0
 #endif
 #ifndef PBA_EXP_EMU_EVERY_D64
 #define PBA_EXP_EMU_EVERY_D64 0
