@@ -428,12 +428,13 @@ def main():
     line["backward"] = run_bwd(args, pba, dev, stream, pg, peaks)
     line["ring8k"] = run_ring8k(args, pba, dev, stream, pg, peaks)
     line["f32"] = run_f32(args, pba, dev, stream, pg, peaks)
+    line["configs"] = run_configs(args, pba, dev, stream, pg, peaks, line, clk)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, pba, cfg, q, k, v, bias, mask, out, lse, stream, pg, world, flops)
     if not args.no_cpu and rank == 0 and world == 1:
         val, cores, desc, secs = oracle_sample(q, k, v, bias, mask, target_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
-                                "seconds": secs}
+                                "seconds": secs, "per_config": oracle_per_config(dev, val, cores)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg:
@@ -638,6 +639,173 @@ def run_f32(args, pba, dev, stream, pg, peaks):
                          "frac": 3 * alg / peak, "kernel": "pba_attn_tf32_sm100_kernel (pba_forward, fp32)",
                          "peak_source": peaks["source"] + " bf16 x 1.1/2.25",
                          "note": "achieved = tf32 tensor-core work, 3x the algorithmic FLOPs"}}
+
+
+def per_call_ms(call, n, stream, pg, flush=None):
+    """Median over n calls of one call's CUDA-event time on the stream, after
+    3 warm-up calls.  With `flush` (a buffer larger than L2) rewritten before
+    each call, no input is left in L2 by the call before."""
+    for _ in range(3):
+        call()
+    barrier(pg)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i, (s, e) in enumerate(ev):
+        if flush is not None:
+            flush.fill_(i & 0xFF)
+        s.record(stream)
+        call()
+        e.record(stream)
+    barrier(pg)
+    return max_over_ranks(statistics.median(s.elapsed_time(e) for s, e in ev), pg)
+
+
+def run_configs(args, pba, dev, stream, pg, peaks, line, clk):
+    """Each workload of the benchmark plan on its own: ms per call (median of
+    20 calls, each after a 256 MB L2 flush), TFLOP/s, GB/s and the roofline
+    fraction; for triangle attention also pair-tensor rows/s (lines of the
+    pair tensor) and softmax rows/s (one per line, query and head).  pr1,
+    apb2k and tri512 are timed here; ring8k, large16k and tri1024 repeat the
+    figures of their own entries of the line."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    n = 20
+    res = {}
+
+    # pr1: fp32, one pass and the four 64-key blocks merged
+    cfg = W.PR1
+    q, k, v, b, _ = W.attn_inputs(cfg, dev)
+    B, H, N, D, P = cfg.B, cfg.H, cfg.N, cfg.D, cfg.blocks
+    out, lse = torch.empty_like(q), torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ms = per_call_ms(lambda: pba.pba_forward(q, k, v, b, None, out, lse, stream=stream), n, stream, pg, flush)
+    L = N // P
+    o_p = torch.empty((P, B, H, N, D), dtype=torch.float32, device=dev)
+    m_p, l_p = torch.empty((P, B, H, N), dtype=torch.float32, device=dev), torch.empty((P, B, H, N), dtype=torch.float32, device=dev)
+    mout, mlse = torch.empty_like(out), torch.empty_like(lse)
+    views = [(k[:, :, j * L:(j + 1) * L], v[:, :, j * L:(j + 1) * L], b[..., j * L:(j + 1) * L]) for j in W.block_order(cfg)]
+
+    def blocks():
+        for slot, (kb, vb, bb) in enumerate(views):
+            pba.pba_partial(q, kb, vb, bb, None, o_p[slot], m_p[slot], l_p[slot], stream=stream)
+        pba.softmax_merge(o_p, m_p, l_p, out_dtype=torch.float32, out=mout, lse=mlse, stream=stream)
+
+    ms_blocks = per_call_ms(blocks, n, stream, pg, flush)
+    flops = attn_flops(B, H, N, N, D)
+    res["pr1"] = {"ms_per_call": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                  "gbs": attn_bytes(B, H, N, N, D, elt=4, mask=False) / (ms / 1e3) / 1e9,
+                  "ms_4_blocks_and_merge": ms_blocks, "gpu_launches_per_call": 1,
+                  "bound": "launch (one wave of 8 CTAs; the roofline floors are below 2 us)",
+                  "workload": "pr1: fp32 N=256 H=4 D=32, no mask; also 4 key blocks of 64 in seeded order + merge"}
+    del q, k, v, b, out, lse, o_p, m_p, l_p, mout, mlse, views
+
+    # apb2k: bf16, last 10 % of the keys masked
+    cfg = W.APB2K
+    q, k, v, b, mask = W.attn_inputs(cfg, dev)
+    B, H, N, D = cfg.B, cfg.H, cfg.N, cfg.D
+    out, lse = torch.empty_like(q), torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ms = per_call_ms(lambda: pba.pba_forward(q, k, v, b, mask, out, lse, stream=stream), n, stream, pg, flush)
+    flops, nbytes = attn_flops(B, H, N, N, D), attn_bytes(B, H, N, N, D)
+    n_valid = int(mask[0].sum().item())
+    res["apb2k"] = {"ms_per_call": ms, "tflops": flops / (ms / 1e3) / 1e12,
+                    "tflops_valid_keys": flops * n_valid / N / (ms / 1e3) / 1e12, "valid_keys": n_valid,
+                    "gbs": nbytes / (ms / 1e3) / 1e9,
+                    "roofline": roofline_entry(flops, nbytes, ms / 1e3, peaks, None, "pba_attn_sm100_kernel (pba_forward, apb2k)"),
+                    "workload": "apb2k: bf16 N=2048 H=16 D=64, bias ~N(0,2), last 204 keys masked"}
+    del q, k, v, b, mask, out, lse
+
+    # tri512: both orientations, gate on
+    tcfg = W.TRI512
+    tq, tk, tv, tg, tb = W.tri_inputs(tcfg, dev)
+    tout = torch.empty_like(tq)
+    tlse = torch.empty((tcfg.N, tcfg.N, tcfg.H), dtype=torch.float32, device=dev)
+    sm_mhz = (clk.get("sm_mhz") or 1965.0) if isinstance(clk, dict) else 1965.0
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tri = {}
+    for orient in ("starting", "ending"):
+        ms = per_call_ms(lambda: pba.tri_attn_forward(tq, tk, tv, tb, tg, None, orient, tout, tlse, stream=stream),
+                         n, stream, pg, flush)
+        tri[orient] = tri_ceilings(tcfg.N, tcfg.H, tcfg.D, ms, peaks["bf16_tflops_sustained"], peaks["hbm_gbs"],
+                                   sm_mhz, n_sms)
+        tri[orient]["pair_rows_per_s"] = tcfg.N / (ms / 1e3)
+        tri[orient]["softmax_rows_per_s"] = tcfg.N * tcfg.N * tcfg.H / (ms / 1e3)
+        tri[orient]["tflops"] = tri[orient]["flops_per_call"] / (ms / 1e3) / 1e12
+    tri["workload"] = "tri512: pair tensor N=512 c=128, H=4 D=32 bf16, gate on, no pair mask"
+    res["tri512"] = tri
+    del tq, tk, tv, tg, tb, tout, tlse
+
+    r8 = line.get("ring8k", {})
+    res["ring8k"] = {k2: r8.get(k2) for k2 in ("partials_ms", "merge_ms_l2_flushed", "pba_forward_ms_same_shape",
+                                               "partials_tflops")}
+    res["ring8k"]["partials_frac"] = r8.get("partials_roofline", {}).get("frac")
+    res["ring8k"]["merge_frac"] = r8.get("merge_roofline", {}).get("frac")
+    rl = line["roofline"]
+    res["large16k"] = {"ms_per_call": line["pba_ms_per_launch"], "tflops": line["value"],
+                       "gbs": rl["hbm_frac"] * peaks["hbm_gbs"], "frac": rl["frac"], "bound": rl["bound"]}
+    t1 = W.TRI1024
+    ms = line["tri_attn_ms_per_call"]
+    res["tri1024"] = {"ms_per_call": ms, "tflops": line["tri_attn_ceilings"]["flops_per_call"] / (ms / 1e3) / 1e12,
+                      "pair_rows_per_s": t1.N / (ms / 1e3), "softmax_rows_per_s": t1.N * t1.N * t1.H / (ms / 1e3),
+                      "frac": line["tri_attn_ceilings"]["frac"]}
+    res["timing"] = f"median of {n} calls, CUDA events, 256 MB L2 flush before each call (pr1, apb2k, tri512)"
+    if pba.pba_last_device_error(stream) != pba.PBA_OK:
+        raise RuntimeError("a kernel recorded a device error in the per-workload timings")
+    return res
+
+
+def oracle_per_config(dev, large_tflops, large_cores):
+    """The fp64 oracle's rate on every workload of the benchmark plan, in
+    softmax rows per second (a row = one query of one head, against all its
+    keys), on the host cores: pr1 and apb2k in full, the others on seeded
+    samples that include the tile-boundary rows (ring8k 512 query rows of
+    every head, tri512 16 lines, tri1024 8 lines); large16k from the
+    cpu_baseline sample.  Inputs are converted to fp64 before each timed
+    call.  The full-size time of a sampled workload is extrapolated and
+    labelled so."""
+    import numpy as np
+
+    import oracle
+
+    f64 = lambda t: np.ascontiguousarray(t.detach().cpu().double().numpy())
+    u8 = lambda t: None if t is None else np.ascontiguousarray(t.detach().cpu().numpy().astype(np.uint8))
+    res = {}
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    for cfg in (W.PR1, W.APB2K, W.RING8K):
+        q, k, v, b, mask = W.attn_inputs(cfg, dev)
+        B, H, N = cfg.B, cfg.H, cfg.N
+        if cfg is W.RING8K:
+            rows = torch.as_tensor(W.sample_rows(N, 512, seed=3), device=dev)
+            q, b = q.index_select(2, rows), b.index_select(2, rows)
+        args = (f64(q), f64(k), f64(v), f64(b), u8(mask))
+        nrows = B * H * args[0].shape[2]
+        t = timed(lambda: oracle.pba(*args))
+        e = {"softmax_rows_per_s": nrows / t, "rows": nrows, "seconds": t}
+        if cfg is W.RING8K:
+            e["extrapolated_full_s"] = B * H * N * t / nrows
+            e["sample"] = "512 query rows (incl. 0, 127, 128, 255, 8191) of every head, all 8192 keys"
+        else:
+            e["sample"] = "full"
+        res[cfg.name] = e
+        del q, k, v, b, mask, args
+    for tcfg, count in ((W.TRI512, 16), (W.TRI1024, 8)):
+        tq, tk, tv, tg, tb = W.tri_inputs(tcfg, dev)
+        lines = torch.as_tensor(W.sample_rows(tcfg.N, count, seed=tcfg.seed), device=dev)
+        sel = lambda x: f64(x.index_select(0, lines))
+        args = (sel(tq), sel(tk), sel(tv), f64(tb), sel(tg))
+        t = timed(lambda: oracle.tri_attn_lines(*args))
+        nrows = count * tcfg.N * tcfg.H
+        res[tcfg.name] = {"softmax_rows_per_s": nrows / t, "pair_rows_per_s": count / t, "rows": nrows,
+                          "seconds": t, "extrapolated_full_s_per_orientation": tcfg.N * t / count,
+                          "sample": f"{count} starting-node lines (incl. 0, 127, 128, 255, {tcfg.N - 1})"}
+        del tq, tk, tv, tg, tb, args
+    L = W.LARGE16K
+    res["large16k"] = {"softmax_rows_per_s": large_tflops * 1e12 / (4.0 * L.N * L.D),
+                       "extrapolated_full_s": L.B * L.H * L.N * 4.0 * L.N * L.D / (large_tflops * 1e12),
+                       "sample": "the cpu_baseline sample"}
+    res["cores"] = large_cores
+    return res
 
 
 def merge_bytes(P, rows, D, out_elt=2):
