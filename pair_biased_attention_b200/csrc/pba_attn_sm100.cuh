@@ -656,6 +656,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       }
 
       // -------------------------------------------------------------- epilogue
+      // What does not need O is done before waiting for the last P V: the
+      // unit's coordinates, 1/l and, with a gate at D = 32 and the
+      // untransposed bias tile, the column factors sigmoid(g) / l of the row
+      // (the exp2 unit works on them while the last P V runs; triangle
+      // attention, starting node, 1.97 -> 1.84 ms at N = 1024).  The other
+      // gated instances form the factors after reading O: there the early
+      // factors add register spills (the ending node measured slower with
+      // them, 1.91 -> 1.94 ms).
+      const Unit un = decode_unit(p, u);  // derived here so it is not live across the tile loop
+      const int row = un.q0 + w * kBM + t;
+      const int b = un.b, h = un.h;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      constexpr bool kEarlyGate = kGate && !kBiasT && D == 32;
+      float sc[kGate ? D : 1];
+      auto gate_factors = [&]() {
+        const uint4 *gptr = reinterpret_cast<const uint4 *>(p.gate + b * p.gate_sb + h * p.gate_sh +
+                                                            (int64_t)row * p.gate_sn);
+        const uint8_t *grow_s = smem + L::kOffOut + (w * kBM + t) * L::kRowBytes;
+        if (L::kOutStaged) cp_async_wait_all();
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 gv = L::kOutStaged ? *reinterpret_cast<const uint4 *>(grow_s + ((c ^ ((t >> 1) & 3)) << 4))
+                                         : gptr[c];
+          const uint32_t wv[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            sc[c * 8 + 2 * e] = inv_l * sigmoid_fast(bf16lo_to_f32(wv[e]));
+            sc[c * 8 + 2 * e + 1] = inv_l * sigmoid_fast(bf16hi_to_f32(wv[e]));
+          }
+        }
+      };
+      if (kEpi == kEpiForward && kEarlyGate && row < p.Nq) gate_factors();
       if (ok) ok = mbar_wait<false>(&bars[L::kBarODone + w], (gt - 1) & 1, wc);
       if (!ok) break;
       tc_fence_after_sync();
@@ -672,9 +704,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       // O is in registers: the next unit's first P V may overwrite it
       tc_fence_before_sync();
       mbar_arrive(&bars[L::kBarOFree + w]);
-      const Unit un = decode_unit(p, u);  // derived here so it is not live across the tile loop
-      const int row = un.q0 + w * kBM + t;
-      const int b = un.b, h = un.h;
       if (kEpi == kEpiForward && L::kOutStaged && !kGate) {
         // the warp's staging rows were last read by the previous unit's store
         // (with a gate this was waited for at the unit's start)
@@ -682,26 +711,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         __syncwarp();
       }
       if (row < p.Nq) {
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
         if (kEpi == kEpiForward) {
-          float g[D];
-          if (kGate) {
-            const uint4 *gptr = reinterpret_cast<const uint4 *>(p.gate + b * p.gate_sb + h * p.gate_sh +
-                                                                (int64_t)row * p.gate_sn);
-            uint8_t *grow_s = smem + L::kOffOut + (w * kBM + t) * L::kRowBytes;
-            if (L::kOutStaged) cp_async_wait_all();
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-              const uint4 gv = L::kOutStaged ? *reinterpret_cast<const uint4 *>(grow_s + ((c ^ ((t >> 1) & 3)) << 4))
-                                             : gptr[c];
-              const uint32_t wv[4] = {gv.x, gv.y, gv.z, gv.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                g[c * 8 + 2 * e] = bf16lo_to_f32(wv[e]);
-                g[c * 8 + 2 * e + 1] = bf16hi_to_f32(wv[e]);
-              }
-            }
-          }
+          if (kGate && !kEarlyGate) gate_factors();
           uint4 *op = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + b * p.out_sb + h * p.out_sh +
                                                 (int64_t)row * p.out_sn);
           // staged rows: this thread's row of the warpgroup's buffer, 16-byte
@@ -712,12 +723,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
             uint32_t wv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              float v0 = o[c * 8 + 2 * e] * inv_l, v1 = o[c * 8 + 2 * e + 1] * inv_l;
-              if (kGate) {
-                v0 *= sigmoid_fast(g[c * 8 + 2 * e]);
-                v1 *= sigmoid_fast(g[c * 8 + 2 * e + 1]);
-              }
-              wv[e] = pack_bf16x2(v0, v1);
+              const int i = c * 8 + 2 * e;
+              wv[e] = kGate ? pack_bf16x2(o[i] * sc[kGate ? i : 0], o[i + 1] * sc[kGate ? i + 1 : 0])
+                            : pack_bf16x2(o[i] * inv_l, o[i + 1] * inv_l);
             }
             if (L::kOutStaged)
               *reinterpret_cast<uint4 *>(srow + ((c ^ ((t >> 1) & 3)) << 4)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
