@@ -517,23 +517,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
       }
       for (int j = 0; j < nt && ok; ++j, ++gt) {
         // The bias tile lands long before it is used: wait for it first and
-        // start loading its first half from shared memory, so that those loads
+        // start loading its first part from shared memory, so that those loads
         // overlap the wait for the score tile and its Tensor Memory load.
         const int slot = w * kBiasStages + (gt % kBiasStages);
         ok = mbar_wait<false>(&bars[(relay ? L::kBarBiasReady : L::kBarBiasFull) + slot], (gt / kBiasStages) & 1, wc);
         if (!ok) break;
         const uint8_t *tile = smem + L::kOffBias + slot * L::kBiasBytes;
-        constexpr int kPre = kBN / 16;  // 8-key groups loaded ahead
+        // 8-key groups of the untransposed tile loaded ahead: half the tile
+        // at D = 64, ten of sixteen at D = 32, where the registers allow it
+        // (triangle attention, starting node, 1.838 -> 1.802 ms at N = 1024;
+        // twelve groups 1.804 ms, and large16k gains nothing from ten)
+        constexpr int kPre = (D == 32) ? 10 : kBN / 16;
+        constexpr int kPreT = 32;        // keys of the transposed tile loaded ahead
         uint4 bpre[kPre];                // untransposed tile: 8 bf16 per group
-        uint32_t tpre[kBiasT ? 4 * kPre : 1];  // transposed tile: 1 bf16 per key
+        uint32_t tpre[kBiasT ? kPreT : 1];  // transposed tile: 1 bf16 per key
         if (kBiasT) {
           const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
 #pragma unroll
-          for (int c = 0; c < 4 * kPre; ++c) tpre[c] = col[c * kBM];
+          for (int c = 0; c < kPreT; ++c) tpre[c] = col[c * kBM];
         } else {
 #pragma unroll
           for (int c8 = 0; c8 < kPre; ++c8)
-            bpre[c8] = *reinterpret_cast<const uint4 *>(tile + t * 128 + ((c8 ^ (t & 7)) << 4));
+            bpre[c8] = *reinterpret_cast<const uint4 *>(tile + (c8 >> 3) * (L::kBiasBytes / 2) + t * 128 +
+                                                        (((c8 & 7) ^ (t & 7)) << 4));
         }
         uint4 kpre[kMasked && !kBiasT ? kPre : 1];  // and their mask words
         if (kMasked && !kBiasT) {
@@ -561,8 +567,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
           const uint16_t *col = reinterpret_cast<const uint16_t *>(tile) + t;
 #pragma unroll
           for (int c = 0; c < kBN; c += 2) {
-            const uint32_t b0 = c < 4 * kPre ? tpre[c] : uint32_t(col[c * kBM]);
-            const uint32_t b1 = c + 1 < 4 * kPre ? tpre[c + 1] : uint32_t(col[(c + 1) * kBM]);
+            const uint32_t b0 = c < kPreT ? tpre[c] : uint32_t(col[c * kBM]);
+            const uint32_t b1 = c + 1 < kPreT ? tpre[c + 1] : uint32_t(col[(c + 1) * kBM]);
             const float2 bv = make_float2(__uint_as_float(b0 << 16), __uint_as_float(b1 << 16));
             x[c / 2] = ffma2(make_float2(__uint_as_float(sreg[c]), __uint_as_float(sreg[c + 1])), tau2, bv);
           }
