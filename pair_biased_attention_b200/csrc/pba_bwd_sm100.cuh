@@ -21,10 +21,13 @@
 //
 // One CTA per unit, 384 threads: warps 0-7 two compute warpgroups (row =
 // thread = Tensor Memory lane; warpgroup g takes columns 64g .. 64g+63 of
-// every step), warp 8 the TMA producer, warp 9 Tensor Memory and the MMAs,
-// warps 10-11 idle.  Per step the chain is S, dP -> P, dS -> dQ or dV, dK; the
-// next step's S, dP are issued as soon as both warpgroups have read this
-// step's.  Operand tiles are double-buffered.
+// every step), warp 8 the TMA producer of the operand tiles, warp 9 Tensor
+// Memory and the MMAs, warp 10 the TMA producer of the bias tiles, warp 11
+// idle.  Per step the chain is S, dP -> P, dS -> dQ or dV, dK; the next
+// step's S, dP are issued as soon as both warpgroups have read this step's.
+// Operand tiles are double-buffered; the bias tiles, streamed from HBM and
+// held until the step's compute (and, in A, its dbias store) is done with
+// them, run in their own ring of three.
 #pragma once
 
 #include <cuda.h>
@@ -39,6 +42,7 @@ constexpr int kBwdComputeGroups = 2;  // column halves of a step, one warpgroup 
 constexpr int kBwdThreads = 128 * (kBwdComputeGroups + 1);
 constexpr int kBwdWarpProducer = 4 * kBwdComputeGroups;
 constexpr int kBwdWarpMma = kBwdWarpProducer + 1;
+constexpr int kBwdWarpBiasProducer = kBwdWarpProducer + 2;
 // Per-thread register limits after the warpgroup reallocation: the launch
 // gives 168 (384 x 168 = 64512); the producer/MMA warpgroup keeps 56 and the
 // compute warpgroups take 224 (128 x 56 + 256 x 224 = 64512).
@@ -78,24 +82,30 @@ struct BwdLayout {
   static constexpr int kAtomBytes = 8 * kRowBytes;
   static constexpr int kTileBytes = kBwdTile * kRowBytes;  // one [128][D] bf16 tile
   static constexpr int kBiasBytes = kBwdTile * kBwdTile * 2;
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 2;      // operand tiles (A: K, V; B: Q, dO)
+  // bias tiles: a third stage gives each HBM load a step more of lead
+  // (ring8k shapes: 2.20 -> 2.02 ms per backward call)
+  static constexpr int kBiasStages = 3;
   // fixed operands of the unit (A: Q, dO; B: K, V), then per-step operands
-  // (A: K, V; B: Q, dO) and the bias tile, double-buffered
+  // (A: K, V; B: Q, dO), double-buffered, and the bias tiles in a ring of
+  // three
   static constexpr int kOffFix0 = 0;
   static constexpr int kOffFix1 = kOffFix0 + kTileBytes;
   static constexpr int kOffStep0 = kOffFix1 + kTileBytes;                   // [stage]
   static constexpr int kOffStep1 = kOffStep0 + kStages * kTileBytes;        // [stage]
-  static constexpr int kOffBias = kOffStep1 + kStages * kTileBytes;         // [stage]
+  static constexpr int kOffBias = kOffStep1 + kStages * kTileBytes;         // [bias stage]
   // per-step column data, one copy per compute warp (so that a warp needs no
   // barrier with the others of its warpgroup), double-buffered by step
   // parity: A: 32 keep words; B: -lse log2(e) and -Delta of 64 query columns
   static constexpr int kRowvWarpFloats = kBwdTile;
-  static constexpr int kOffRowv = kOffBias + kStages * kBiasBytes;
+  static constexpr int kOffRowv = kOffBias + kBiasStages * kBiasBytes;
   static constexpr int kOffBar = kOffRowv + 2 * (4 * kBwdComputeGroups) * kRowvWarpFloats * 4;
   static constexpr int kBarFixFull = 0;
   static constexpr int kBarStepFull = 1;                       // [stage]
   static constexpr int kBarStepEmpty = kBarStepFull + kStages;  // [stage]
-  static constexpr int kBarSFull = kBarStepEmpty + kStages;
+  static constexpr int kBarBiasFull = kBarStepEmpty + kStages;       // [bias stage]
+  static constexpr int kBarBiasEmpty = kBarBiasFull + kBiasStages;   // [bias stage]
+  static constexpr int kBarSFull = kBarBiasEmpty + kBiasStages;
   static constexpr int kBarSFree = kBarSFull + 1;
   static constexpr int kBarGFull = kBarSFree + 1;  // P / dS written to Tensor Memory
   static constexpr int kBarGDone = kBarGFull + 1;  // the accumulating MMAs of a step are done
@@ -137,9 +147,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     mbar_init(&bars[L::kBarFixFull], 1);
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(&bars[L::kBarStepFull + s], 1);
-      // the MMA commit + each compute warp (A: its dbias store has read the
-      // slot) or warpgroup (B: its bias half is read)
-      mbar_init(&bars[L::kBarStepEmpty + s], 1 + (kB ? kBwdComputeGroups : 4 * kBwdComputeGroups));
+      mbar_init(&bars[L::kBarStepEmpty + s], 1);  // the MMA commit after the step's last MMAs
+    }
+    for (int s = 0; s < L::kBiasStages; ++s) {
+      mbar_init(&bars[L::kBarBiasFull + s], 1);
+      // each compute warp (A: once its dbias store has read the slot)
+      mbar_init(&bars[L::kBarBiasEmpty + s], 4 * kBwdComputeGroups);
     }
     mbar_init(&bars[L::kBarSFull], 1);
     mbar_init(&bars[L::kBarSFree], kBwdComputeGroups * kBwdTile);
@@ -180,11 +193,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
           if (!ok) break;
           const int o0 = it * kBwdTile;
           uint64_t *full = &bars[L::kBarStepFull + s];
-          mbar_arrive_expect_tx(full, 2 * L::kTileBytes + L::kBiasBytes);
+          mbar_arrive_expect_tx(full, 2 * L::kTileBytes);
           tma_load_4d(smem + L::kOffStep0 + s * L::kTileBytes, kB ? &p.tm_q : &p.tm_k, full, 0, o0, h, b, pol);
           tma_load_4d(smem + L::kOffStep1 + s * L::kTileBytes, kB ? &p.tm_do : &p.tm_v, full, 0, o0, h, b, pol);
+        }
+        mbar_wait(&bars[L::kBarFixFull], 0, wc_drain);
+        if (!ok)
+          for (int s = 0; s < L::kStages; ++s) {
+            const int a = (it - s + L::kStages - 1) / L::kStages;
+            if (a > 0) mbar_wait(&bars[L::kBarStepFull + s], (a - 1) & 1, wc_drain);
+          }
+      }
+    } else if (warp == kBwdWarpBiasProducer) {
+      // ================================================================ bias tiles
+      if (lane == 0) {
+        const uint64_t pol = l2_policy_evict_last();
+        const int hb = p.bias_h_bcast ? 0 : h, bb = p.bias_b_bcast ? 0 : b;
+        bool ok = true;
+        int it = 0;
+        for (; it < nsteps && ok; ++it) {
+          const int s = it % L::kBiasStages;
+          if (it >= L::kBiasStages)
+            ok = mbar_wait(&bars[L::kBarBiasEmpty + s], ((it / L::kBiasStages) - 1) & 1, wc);
+          if (!ok) break;
+          const int o0 = it * kBwdTile;
+          uint64_t *full = &bars[L::kBarBiasFull + s];
           uint8_t *bdst = smem + L::kOffBias + s * L::kBiasBytes;
-          const int hb = p.bias_h_bcast ? 0 : h, bb = p.bias_b_bcast ? 0 : b;
+          mbar_arrive_expect_tx(full, L::kBiasBytes);
           if (kB) {
             // [128 queries][128 keys], no swizzle: the thread of key j reads column j
             tma_load_4d(bdst, &p.tm_bias, full, row0, o0, hb, bb, pol);
@@ -194,11 +229,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
             tma_load_4d(bdst + L::kBiasBytes / 2, &p.tm_bias, full, o0 + 64, row0, hb, bb, pol);
           }
         }
-        mbar_wait(&bars[L::kBarFixFull], 0, wc_drain);
         if (!ok)
-          for (int s = 0; s < L::kStages; ++s) {
-            const int a = (it - s + L::kStages - 1) / L::kStages;
-            if (a > 0) mbar_wait(&bars[L::kBarStepFull + s], (a - 1) & 1, wc_drain);
+          for (int s = 0; s < L::kBiasStages; ++s) {
+            const int a = (it - s + L::kBiasStages - 1) / L::kBiasStages;
+            if (a > 0) mbar_wait(&bars[L::kBarBiasFull + s], (a - 1) & 1, wc_drain);
           }
       }
     } else if (warp == kBwdWarpMma) {
@@ -322,17 +356,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
     };
     if (nsteps > 0) load_cols(0);
     bool ok = true;
+    uint32_t bias_off = 0, bias_ph = 0;  // the step's bias slot (bytes) and its phase
     for (int it = 0; it < nsteps && ok; ++it) {
-      const int s = it % L::kStages;
       const int o0 = it * kBwdTile;
       const uint32_t cm0 = nm0, cm1 = nm1;
       const float clse[2] = {nlse[0], nlse[1]}, cdelta[2] = {ndelta[0], ndelta[1]};
       if (it + 1 < nsteps) load_cols(it + 1);
-      // S, dP and the step's tiles.  The waits only set ok; the warp leaves
-      // together at the vote below.
+      // S, dP and the step's bias tile.  The waits only set ok; the warp
+      // leaves together at the vote below.
+      const int bs = bias_off / L::kBiasBytes;
       ok = mbar_wait<false>(&bars[L::kBarSFull], it & 1, wc);
-      if (ok) ok = mbar_wait<false>(&bars[L::kBarStepFull + s], (it / L::kStages) & 1, wc);
-      const uint8_t *bt = smem + L::kOffBias + s * L::kBiasBytes;
+      if (ok) ok = mbar_wait<false>(&bars[L::kBarBiasFull + bs], bias_ph, wc);
+      const uint8_t *bt = smem + L::kOffBias + bias_off;
       // Per-step column data in this warp's own shared-memory copy
       // (double-buffered by step parity), written and read by the warp alone.
       // A: one keep word per key pair of the warpgroup's 64 columns (0xFFFF
@@ -483,10 +518,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
                        b);
           bulk_commit_group();
           bulk_wait_group_read<0>();
-          mbar_arrive(&bars[L::kBarStepEmpty + s]);
+          mbar_arrive(&bars[L::kBarBiasEmpty + bias_off / L::kBiasBytes]);
         }
-      } else if (t == 0) {
-        mbar_arrive(&bars[L::kBarStepEmpty + s]);  // this warpgroup's bias half read
+      } else {
+        // this warp's reads of the bias slot are done
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[L::kBarBiasEmpty + bias_off / L::kBiasBytes]);
+      }
+      bias_off += L::kBiasBytes;
+      if (bias_off == uint32_t(L::kBiasStages * L::kBiasBytes)) {
+        bias_off = 0;
+        bias_ph ^= 1u;
       }
     }
     // -------------------------------------------------------------- epilogue
