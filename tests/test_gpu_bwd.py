@@ -82,6 +82,7 @@ def _run(name, q, k, v, bias, mask, seed=0, scale=None):
     (2, 3, 200, 264, 64, 0.1),     # ragged query and key tiles, mask
     (1, 2, 384, 256, 32, 0.2),     # D = 32, several tiles
     (1, 1, 64, 512, 64, 0.5),      # half the keys masked
+    (1, 2, 130, 1000, 32, 0.1),    # eight key steps with a ragged last one (the bias ring wraps twice)
 ])
 def test_backward_shapes(cuda_device, B, H, Nq, Nk, D, mask_frac):
     q, k, v, bias, mask = W.random_attn(B, H, Nq, Nk, D, seed=Nq + Nk + D, device=cuda_device, mask_frac=mask_frac)
