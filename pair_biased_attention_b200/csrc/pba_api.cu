@@ -603,12 +603,13 @@ pba_status softmax_merge(int32_t P, int64_t rows, int64_t D, const float *o_part
   if (s != PBA_OK) return s;
   if (rows == 0) return PBA_OK;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t total = rows * (D / 4);
   int64_t grid = (total + 255) / 256;
-  const int64_t cap = int64_t(sms) * 8;  // a few resident blocks per SM, grid-stride beyond
+  // One thread per 4-element chunk: blocks that finish make room for new
+  // ones, whose loads overlap the others' arithmetic (ring8k merge 57.3 ->
+  // 53.2 us against a grid of 8 blocks per SM looping over the rows).  The
+  // kernel's grid-stride loop covers sizes beyond the cap.
+  const int64_t cap = int64_t(1) << 30;
   if (grid > cap) grid = cap;
   const bool bf = out_dtype == PBA_BF16;
   // P up to 8 (the ring steps of one node) unrolled with all loads up front; larger P loops
