@@ -922,7 +922,7 @@ pba_status pba_backward(const pba_attn_desc *d, const void *q, const void *k, co
   p.timeout_ns = g_timeout_ns.load();
   // Delta = rowsum(dO * O)
   const int64_t rows = B * H * Nq;
-  pba::pba_bwd_delta_kernel<<<int((rows * 32 + 255) / 256), 256, 0, st>>>(
+  pba::pba_bwd_delta_kernel<<<int((rows * (D / 8) + 255) / 256), 256, 0, st>>>(
       static_cast<const uint16_t *>(dout), static_cast<const uint16_t *>(out), delta, rows, int(D));
   if (cudaGetLastError() != cudaSuccess) return PBA_ERR_CUDA;
   cudaError_t e;

@@ -573,17 +573,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) pba_bwd_sm100_kernel(const __g
   if (warp == kBwdWarpMma) tmem_dealloc(tmem, 512);
 }
 
-// Delta_i = sum_d dO_id O_id (bf16 inputs, fp32 sum), one warp per row.
+// Delta_i = sum_d dO_id O_id (bf16 inputs, fp32 sum).  D / 8 lanes per row
+// (D = 32 or 64), each with one 16-byte load of dO and of O (8 features); the
+// lanes of a row add their sums by shuffles.  dO and O are contiguous
+// [rows][D] bf16 rows starting on 16-byte boundaries.
 __global__ void pba_bwd_delta_kernel(const uint16_t *dout, const uint16_t *out, float *delta, int64_t rows, int D) {
-  const int64_t row = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
+  const int lpr = D >> 3;  // lanes per row, a divisor of 32
+  const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t row = t / lpr;
+  const int c = int(t - row * lpr);
   float acc = 0.f;
-  for (int d = lane; d < D; d += 32)
-    acc += __uint_as_float(uint32_t(dout[row * D + d]) << 16) * __uint_as_float(uint32_t(out[row * D + d]) << 16);
+  if (row < rows) {
+    const uint4 a = reinterpret_cast<const uint4 *>(dout + row * D)[c];
+    const uint4 b = reinterpret_cast<const uint4 *>(out + row * D)[c];
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) delta[row] = acc;
+    for (int e = 0; e < 4; ++e)
+      acc += __uint_as_float(aw[e] << 16) * __uint_as_float(bw[e] << 16) +
+             __uint_as_float(aw[e] & 0xFFFF0000u) * __uint_as_float(bw[e] & 0xFFFF0000u);
+  }
+  // every lane of the warp takes part; rows past the end add zeros
+  for (int o = lpr >> 1; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (row < rows && c == 0) delta[row] = acc;
 }
 
 }  // namespace pba
