@@ -337,6 +337,24 @@ def test_merge_edge_cases(cuda_device):
     assert (mo - o_parts[0]).abs().max().item() < 1e-6
 
 
+@pytest.mark.parametrize("P,rows,D", [(11, 777, 32), (16, 300, 64), (3, 5, 32)])
+def test_merge_many_blocks_and_ragged_rows(cuda_device, P, rows, D):
+    """More partials than the unrolled kernels take (P > 8: the looping
+    kernel), a row count that leaves the last block of threads part-filled,
+    and very few rows; one block of every row empty."""
+    g = torch.Generator("cuda").manual_seed(P * 100 + rows)
+    o_parts = torch.randn((P, rows, D), generator=g, device=cuda_device)
+    m_parts = torch.randn((P, rows), generator=g, device=cuda_device) * 4
+    l_parts = torch.rand((P, rows), generator=g, device=cuda_device) * 10 + 0.1
+    empty = torch.arange(rows, device=cuda_device) % P
+    l_parts[empty, torch.arange(rows, device=cuda_device)] = 0
+    m_parts[empty, torch.arange(rows, device=cuda_device)] = -math.inf
+    ref = oracle.merge(o_parts, m_parts, l_parts)
+    for dt in (torch.float32, torch.bfloat16):
+        mo, ml = pba.softmax_merge(o_parts, m_parts, l_parts, out_dtype=dt)
+        _cmp(f"merge P={P} rows={rows} D={D} {dt}", mo, ml, ref, out_tol=OUT_TOL if dt == torch.bfloat16 else 1e-5)
+
+
 # ------------------------------------------------------------------ bit-exact integer / index handling
 def test_bitexact_masked_entries_do_not_matter(cuda_device):
     q, k, v, bias, mask = W.random_attn(1, 4, 500, 777, 64, seed=11, device=cuda_device, mask_frac=0.3)
