@@ -559,13 +559,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) pba_attn_sm100_kernel(const _
         reg_fence(sreg);
         tc_fence_before_sync();
         // The score tile is free once it is in registers.  The ending node
-        // (transposed bias tile, 128 column loads per thread) frees it only
-        // after its bias loads have returned (with the bias slot, below), so
-        // that the next score MMAs, which stream their operands from shared
-        // memory, do not starve those loads: tri1024 ending node 1.900 ->
-        // 1.879 ms.  The untransposed tile, prefetched ahead, measured
-        // slower that way (1.804 -> 1.823 ms starting node).
-        constexpr bool kLateSFree = kBiasT;
+        // (transposed bias tile, 128 column loads per thread) and D = 64
+        // (half the bias tile and its mask words still to load) free it only
+        // after their bias loads have returned (with the bias slot, below),
+        // so that the next score MMAs, which stream their operands from
+        // shared memory, do not starve those loads: tri1024 ending node
+        // 1.900 -> 1.879 ms, large16k 2.062 -> 2.053 ms.  The starting node
+        // at D = 32, with most of its tile loaded ahead, measured slower that
+        // way (1.804 -> 1.823 ms).
+        constexpr bool kLateSFree = kBiasT || D == 64;
         if (!kLateSFree) mbar_arrive(&bars[L::kBarSFree + w]);
 
         // x = tau * s + bias, two keys per packed fma
